@@ -1,0 +1,337 @@
+"""Benchmark: one SMC-SD round (score -> resample -> page-table remap) per step.
+
+Workload: 256 sequences x 32 particles x (8+1) positions, V = 128256, bf16
+target and draft logits (~37.8 GB read per round), systematic resampling and
+a 128-page table remap for all 8192 particles.  Inputs are synthetic (seeded
+generator, built on the device) and larger than L2, so no flush is needed.
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under torchrun;
+each rank runs its own replica of the workload on disjoint sequences (weak
+scaling, no collective on the data path; barrier + max-over-ranks timing).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "verify+resample logit rows/s; achieved HBM TB/s as fraction of B200 peak"
+WORKLOAD = "smc_scale"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _oracle_sequence(cfg, b):
+    from synth import gen
+    h = gen.gen_config_rows(cfg, seqs=[b])
+    pt = gen.page_table(cfg.seed, cfg.B, cfg.N, cfg.P)[b:b + 1]
+    return h, pt
+
+
+def _oracle_round(cfg, h, pt, parts):
+    """The oracle's SMC-SD round on particles `parts` of one sequence."""
+    import oracle
+    zT, zD, x = h["zT"][:, parts], h["zD"][:, parts], h["draft"][:, parts]
+    o = oracle.smcsd_score(zT, zD, x, cfg.tau, cfg.seed, 1)
+    r = oracle.smcsd_resample(o["logw"], cfg.seed, 1)
+    p = pt[:, parts]
+    oracle.kv_pagetable_remap(p, r["ancestors"], num_pages=int(pt.size), tok_in=o["tokens"])
+    return len(parts) * cfg.R
+
+
+def oracle_baseline(cfg, budget_s=10.0):
+    """Times the oracle (as it stands, one host core) on one whole sequence of the
+    workload, repeated until the budget is used; returns rows/s, seconds, runs."""
+    h, pt = _oracle_sequence(cfg, 0)
+    rows, t_total, runs = 0, 0.0, 0
+    while runs == 0 or t_total < budget_s:
+        t0 = time.perf_counter()
+        rows += _oracle_round(cfg, h, pt, list(range(cfg.N)))
+        t_total += time.perf_counter() - t0
+        runs += 1
+    return rows / t_total, t_total, runs
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 NumPy oracle on a host core (rank 0 only).
+    One step = the oracle's round on 8 particles (72 row pairs) of one sequence."""
+    if rank != 0:
+        return
+    from synth import gen
+    cfg = gen.CONFIGS[WORKLOAD]
+    h, pt = _oracle_sequence(cfg, 0)
+    groups = [list(range(g, g + 8)) for g in range(0, cfg.N, 8)]
+    for i in range(args.warmup):
+        _oracle_round(cfg, h, pt, groups[i % len(groups)])
+    rows, t_total = 0, 0.0
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        rows += _oracle_round(cfg, h, pt, groups[i % len(groups)])
+        t_total += time.perf_counter() - t0
+    value = rows / t_total
+    sample = (f"per step 8 particles x {cfg.R} row pairs (V={cfg.V}) of sequence 0 of the "
+              f"workload, NumPy fp64, one core")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t_total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": cfg.B, "N": cfg.N, "K": cfg.K, "V": cfg.V,
+                   "logits": cfg.dtype, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    import resample_online_log_b200 as lib
+    from synth import device as sdev
+    from synth import gen
+
+    cfg = gen.CONFIGS[WORKLOAD]
+    if rank:  # disjoint synthetic sequences per replica
+        cfg = gen.SynthConfig(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
+    B, N, R, K, V, P = cfg.B, cfg.N, cfg.R, cfg.K, cfg.V, cfg.P
+    dev = "cuda"
+    d = sdev.gen_config_device(cfg)
+    zT, zD, x = d["zT"], d["zD"], d["draft"]
+    pt = torch.from_numpy(gen.page_table(cfg.seed, B, N, P)).to(dev)
+    logw = torch.empty((B, N), dtype=torch.float64, device=dev)
+    bonus = torch.empty((B, N), dtype=torch.int32, device=dev)
+    tv = torch.empty((B, N, R), dtype=torch.float32, device=dev)
+    toks = torch.empty((B, N, R), dtype=torch.int32, device=dev)
+    anc = torch.empty((B, N), dtype=torch.int32, device=dev)
+    W = torch.empty((B, N), dtype=torch.float64, device=dev)
+    ess = torch.empty((B,), dtype=torch.float64, device=dev)
+    pt_out = torch.empty_like(pt)
+    tok_out = torch.empty_like(toks)
+    refcnt = torch.empty((B * N * P,), dtype=torch.int32, device=dev)
+    err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    ev_pairs = []
+
+    def step(i, record=False):
+        rnd = i + 1
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        lib.smcsd_score(zT, zD, x, cfg.tau, cfg.seed, rnd, logw, bonus, tv_out=tv, tokens_out=toks,
+                        dev_err=err)
+        if record:
+            e1.record(stream)
+            ev_pairs.append((e0, e1))
+        lib.smcsd_resample(logw, cfg.seed, rnd, anc, w_out=W, ess_out=ess, dev_err=err)
+        lib.kv_pagetable_remap(pt, anc, pt_out, tok_in=toks, tok_out=tok_out, page_refcnt=refcnt,
+                               num_pages=B * N * P, dev_err=err)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, record=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms_local, world)
+    score_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_pairs)
+    score_ms = max_over_ranks(score_ms, world)
+    assert int(err.item()) == 0, f"device error word {int(err.item())}"
+
+    rows_per_step = B * N * R
+    value = rows_per_step * world * args.steps / (ms * 1e-3)
+    esize = 2 if cfg.dtype == "bf16" else 4
+    alg_bytes = (2 * rows_per_step * V * esize + B * N * K * 4      # logits + draft tokens
+                 + B * N * (8 + 4) + rows_per_step * (4 + 4))       # logw, bonus, tv, tokens
+    hbm_peak, peak_kind = peaks()
+    achieved = alg_bytes / (score_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "N": N, "K": K, "V": V, "logits": cfg.dtype,
+                   "tau": cfg.tau, "pages_per_particle": P, "parallelism": f"replicas{world}",
+                   "l2": "inputs (37.8 GB) larger than L2; no flush"},
+        "hbm_TBps_score": achieved / 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "score_kernel",
+                     "peak_kind": peak_kind, "score_ms": score_ms,
+                     "algorithmic_bytes": alg_bytes},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    # End to end through the public API with host buffers (pinned), one replica.
+    if args.e2e_steps > 0:
+        h_zT = torch.empty(zT.shape, dtype=zT.dtype, pin_memory=True)
+        h_zD = torch.empty(zD.shape, dtype=zD.dtype, pin_memory=True)
+        h_x = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        h_pt = pt.cpu().pin_memory()
+        h_zT.copy_(zT)
+        h_zD.copy_(zD)
+        h_x.copy_(x)
+        outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                for t in (logw, bonus, anc, pt_out, tok_out)]
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.e2e_steps):
+            zT.copy_(h_zT, non_blocking=True)
+            zD.copy_(h_zD, non_blocking=True)
+            x.copy_(h_x, non_blocking=True)
+            pt.copy_(h_pt, non_blocking=True)
+            step(1000 + i)
+            for o, t in zip(outs, (logw, bonus, anc, pt_out, tok_out)):
+                o.copy_(t, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        h2d = sum(t.numel() * t.element_size() for t in (h_zT, h_zD, h_x, h_pt))
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        line["e2e"] = {"value": rows_per_step * world * args.e2e_steps / (e2e_ms * 1e-3),
+                       "unit": "rows/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "steps": args.e2e_steps}
+        del h_zT, h_zD
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, t, runs = oracle_baseline(gen.CONFIGS[WORKLOAD], budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                                "sample": f"sequence 0 of the workload ({N * R} row pairs) x "
+                                          f"{runs} run(s), {t:.1f} s of CPU"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank, world, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+/*
+ * smcsd.h -- C ABI of libsmcsd.so: the per-round scoring / resampling hot path
+ * shared by SMC speculative decoding, standard speculative-decoding
+ * verification and Gumbel-top-k drafting, for NVIDIA B200 (sm_100a).
+ *
+ * Sources (gist.science summaries; each entry point cites its passage):
+ *   [SMC-SD]  "Faster LLM Inference via Sequential Monte Carlo", section 2
+ *             (Methodology: particles, scoring, importance weights,
+ *             evict/duplicate resampling, bonus token, KV page metadata copy)
+ *             and section 1 (standard SD and its rejection step).
+ *   [METASD]  METASD (multi-drafter speculative decoding), section 2
+ *             (Block Divergence reward built on total-variation distance).
+ *   [STAND]   STAND (stochastic adaptive n-gram drafting), Methodology items
+ *             1 (top-10 logit n-gram store) and 2 (Gumbel-Top-K sampling).
+ *
+ * Conventions for every entry point
+ *   - Pointers marked "device" are caller-owned CUDA device pointers; the
+ *     library never allocates, frees or keeps them.  Logit rows are
+ *     row-major with the vocabulary contiguous; `ld` is the element distance
+ *     between consecutive rows (ld >= V), so a slice of a wider buffer works.
+ *   - `stream` is a cudaStream_t passed as void*; all work is enqueued on it
+ *     and the call returns without synchronising.
+ *   - Arguments are checked on the host before anything is enqueued; a bad
+ *     argument returns SD_ERR_INVALID_ARG and enqueues nothing.  A launch
+ *     failure returns SD_ERR_CUDA.  Sizes beyond what a kernel supports
+ *     return SD_ERR_UNSUPPORTED.
+ *   - Faults found on the device (bad token ids, NaN / +inf / all -inf rows,
+ *     page ids out of range, an internal wait that ran out) never trap: they
+ *     OR bits into *dev_err (device, may be NULL) and mark the affected
+ *     outputs (NaN for reals, -1 for ids).  Read *dev_err after the stream
+ *     has been synchronised; the library never clears it.
+ *   - Randomness is counter-based Philox4x32-10: results are a pure function
+ *     of (inputs, seed, round) and reruns are bit-identical.  Counter layout:
+ *     key = seed; counter = (c0, row id, round mod 2^32,
+ *     stream tag + 16 * ((round >> 32) mod 2^28)); per-vocabulary-entry noise
+ *     uses c0 = entry / 4 and output word entry % 4; per-row draws use
+ *     c0 = 0, word 0.  Uniform u = ((w >> 9) + 1/2) * 2^-23; Gumbel
+ *     g = -log(-log u).
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef SMCSD_H_
+#define SMCSD_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SMCSD_API __attribute__((visibility("default")))
+#else
+#define SMCSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sd_status {
+  SD_OK = 0,
+  SD_ERR_INVALID_ARG = 1,
+  SD_ERR_CUDA = 2,
+  SD_ERR_UNSUPPORTED = 3
+} sd_status;
+
+typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
+
+/* Bits of the device error word. */
+#define SD_DEV_TOKEN_OOB 1u      /* a draft token id outside [0, V)            */
+#define SD_DEV_NONFINITE 2u      /* a row with NaN / +inf, or all -inf         */
+#define SD_DEV_ZERO_RESIDUAL 4u  /* verify: rejection with max(p - q, 0) == 0  */
+#define SD_DEV_PAGE_OOB 8u       /* page id outside [0, num_pages) and != -1   */
+#define SD_DEV_ANCESTOR_OOB 16u  /* ancestor index outside [0, N)              */
+#define SD_DEV_TIMEOUT 32u       /* an internal bounded wait gave up           */
+
+/* Philox stream tags. */
+#define SD_STREAM_BONUS 1u
+#define SD_STREAM_ACCEPT 2u
+#define SD_STREAM_RESIDUAL 3u
+#define SD_STREAM_RESAMPLE 4u
+#define SD_STREAM_TOPK_DENSE 5u
+#define SD_STREAM_TOPK_SPARSE 6u
+
+/*
+ * smcsd_score -- scoring step of one SMC-SD round ([SMC-SD] section 2, scoring
+ * and resampling steps; bonus token; [METASD] section 2 for TV).
+ *
+ * For B sequences x N particles x (K+1) positions, with p = softmax(zT/tau),
+ * q = softmax(zD/tau) per row (the same tau divides both):
+ *   lse       of every target and draft row;
+ *   log-probs lp = log p(x_{k+1}), lq = log q(x_{k+1}) at rows k < K;
+ *   logw[b,n] = logw_prev[b,n] + sum_{k<K} (lp - lq)     (importance weight);
+ *   tv[b,n,k] = 1/2 sum_v |p_v - q_v| at all K+1 rows    (block divergence);
+ *   bonus[b,n] = argmax_v (zT[b,n,K,v]/tau + g_v), g from stream 1 with row
+ *                id b*N+n, ties to the lower v           (bonus token).
+ *
+ * zT, zD        device, [B, N, K+1, V] at row stride ld, dtype dt (fp32 or
+ *               bf16).  Both tensors have K+1 rows per particle.
+ * draft_tokens  device int32 [B, N, K]: token x_{k+1} scored at row k.
+ * tau           > 0, finite.
+ * logw_prev     device fp64 [B, N] or NULL (NULL = 0, i.e. after resampling).
+ * logw_out      device fp64 [B, N]                       (required)
+ * bonus_out     device int32 [B, N]                      (required)
+ * tv_out        device fp32 [B, N, K+1]                  (or NULL)
+ * tokens_out    device int32 [B, N, K+1]: x_1..x_K, bonus (or NULL)
+ * lse_out       device fp64 [B, N, K+1, 2]: (lse target, lse draft) (or NULL)
+ * lp_out        device fp64 [B, N, K, 2]: (lp, lq)       (or NULL)
+ * Requirements: B >= 0 (0 = no-op), N >= 1, K >= 0, 1 <= V <= 262144,
+ *   ld >= V; B*N*(K+1) < 2^31.
+ * Faults: token id outside [0, V) -> SD_DEV_TOKEN_OOB, that particle's lp/lq
+ *   and logw are NaN.  Non-finite row -> SD_DEV_NONFINITE, its lse / tv / lp
+ *   NaN, logw NaN, bonus -1 if it is the bonus row.
+ */
+SMCSD_API sd_status smcsd_score(const void* zT, const void* zD, sd_dtype dt, int B, int N, int K, int V,
+                      int64_t ld, const int32_t* draft_tokens, float tau, uint64_t seed,
+                      uint64_t round, const double* logw_prev, double* logw_out,
+                      int32_t* bonus_out, float* tv_out, int32_t* tokens_out, double* lse_out,
+                      double* lp_out, uint32_t* dev_err, void* stream);
+
+/*
+ * smcsd_resample -- weight normalisation, ESS and systematic resampling
+ * ([SMC-SD] section 2: evict low-weight particles, duplicate high-weight ones;
+ * the scheme is systematic and runs every round).
+ *   W[b,j]   = exp(logw_j - max) / sum_m exp(logw_m - max)       (fp64)
+ *   ess[b]   = 1 / sum_j W_j^2
+ *   anc[b,i] = min{ j : W_0 + ... + W_j > (i + u0)/N }, clamped to N-1,
+ *              u0 = uniform of stream 4, row id b.
+ * logw      device fp64 [B, N]; w_out device fp64 [B, N] (or NULL);
+ * ess_out   device fp64 [B] (or NULL); ancestors_out device int32 [B, N].
+ * Requirements: B >= 0, 1 <= N <= 8192.
+ * Faults: a sequence with NaN / +inf weights, or all -inf -> SD_DEV_NONFINITE,
+ *   W and ess NaN, identity ancestors.
+ */
+SMCSD_API sd_status smcsd_resample(const double* logw, int B, int N, uint64_t seed, uint64_t round,
+                         double* w_out, double* ess_out, int32_t* ancestors_out,
+                         uint32_t* dev_err, void* stream);
+
+/*
+ * kv_pagetable_remap -- KV cache update after resampling by page-pointer /
+ * metadata copy instead of KV tensor copy ([SMC-SD] section 2, KV cache
+ * management).
+ *   pt_out[b,i,:]  = pt_in[b, anc[b,i], :]
+ *   tok_out[b,i,:] = tok_in[b, anc[b,i], :]            (if tok_in != NULL)
+ *   refcnt[p]      = #{ (b,i,s) : pt_out[b,i,s] == p }  (if page_refcnt != NULL;
+ *                    the call zeroes it first)
+ * pt_in, pt_out  device int32 [B, N, P]; must not alias.  -1 = empty slot.
+ * ancestors      device int32 [B, N].
+ * tok_in/tok_out device int32 [B, N, T] (both or neither); T >= 0.
+ * page_refcnt    device int32 [num_pages] or NULL.
+ * Faults: ancestor outside [0, N) -> SD_DEV_ANCESTOR_OOB, that particle's
+ *   rows are filled with -1.  Page id outside [0, num_pages) other than -1
+ *   -> SD_DEV_PAGE_OOB, copied but not counted.
+ */
+SMCSD_API sd_status kv_pagetable_remap(const int32_t* pt_in, const int32_t* ancestors, int B, int N, int P,
+                             int32_t* pt_out, const int32_t* tok_in, int T, int32_t* tok_out,
+                             int32_t* page_refcnt, int num_pages, uint32_t* dev_err,
+                             void* stream);
+
+/*
+ * sd_verify_reject -- standard speculative-decoding verification, N = 1
+ * ([SMC-SD] section 1 and [METASD] section 1: the first rejection discards the
+ * rest; textbook rule below), with per-position TV ([METASD] section 2).
+ *   for k < K: accept x_{k+1} iff u_k * q(x) < p(x), u_k from stream 2,
+ *     row id b*(K+1)+k;  at the first reject j the emitted token is
+ *     argmax_{v : r_v > 0} (log r_v + g_v), r = max(p_j - q_j, 0), g from
+ *     stream 3 with row id b*(K+1)+j;  if all K are accepted the bonus token
+ *     is argmax_v (zT[b,K,v]/tau + g_v), stream 1, row id b.
+ * zT  device [B, K+1, V], zD device [B, K, V], row stride ld, dtype dt.
+ * draft_tokens  device int32 [B, K].
+ * accepted_len  device int32 [B]: j (or K).
+ * out_tokens    device int32 [B, K+1]: accepted drafts, then the drawn token,
+ *               then -1 padding.
+ * tv_out        device fp32 [B, K] or NULL.
+ * Requirements: B >= 0, K >= 1, 1 <= V <= 262144, ld >= V.
+ * Faults: a draft id outside [0, V) is rejected (SD_DEV_TOKEN_OOB); a
+ *   non-finite row reached by the sequence stops it there without a token
+ *   (SD_DEV_NONFINITE); an all-zero residual falls back to sampling p
+ *   (SD_DEV_ZERO_RESIDUAL).
+ */
+SMCSD_API sd_status sd_verify_reject(const void* zT, const void* zD, sd_dtype dt, int B, int K, int V,
+                           int64_t ld, const int32_t* draft_tokens, float tau, uint64_t seed,
+                           uint64_t round, int32_t* accepted_len, int32_t* out_tokens,
+                           float* tv_out, uint32_t* dev_err, void* stream);
+
+/*
+ * gumbel_topk -- k tokens per row without replacement by Gumbel-top-k
+ * ([STAND] Methodology item 2): the k largest s_v + g_v, s = z/tau, g from
+ * stream 5 with row id = row, descending, ties to the lower v.
+ * z          device [rows, V] at row stride ld, dtype dt.
+ * idx_out    device int32 [rows, k] (required).
+ * score_out  device fp32 [rows, k]: s_v + g_v (or NULL).
+ * logp_out   device fp32 [rows, k]: s_v - logsumexp(s) (or NULL).
+ * Requirements: rows >= 0, 1 <= k <= 64, k <= V, ld >= V.
+ * Faults: rows with NaN / +inf or all -inf -> SD_DEV_NONFINITE, ids -1;
+ *   ranks with no finite entry left are -1.
+ */
+SMCSD_API sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, int64_t ld, int k, float tau,
+                      uint64_t seed, uint64_t round, int32_t* idx_out, float* score_out,
+                      float* logp_out, uint32_t* dev_err, void* stream);
+
+/*
+ * gumbel_topk_sparse -- the same draw over stored top-L (index, probability)
+ * rows of a logit n-gram store ([STAND] Methodology items 1-2): s_l =
+ * log(prob_l)/tau (prob 0 = unstored = never drawn), g from stream 6 with row
+ * id = row at stored position l; ties to the lower l; outputs the stored
+ * global ids.
+ * idx   device int32 [rows, L];  prob device fp32 [rows, L];
+ * idx_out device int32 [rows, k].
+ * Requirements: rows >= 0, 1 <= L <= 64, 1 <= k <= L.
+ * Faults: NaN / negative / infinite probability -> SD_DEV_NONFINITE, ids -1.
+ */
+SMCSD_API sd_status gumbel_topk_sparse(const int32_t* idx, const float* prob, int rows, int L, int k,
+                             float tau, uint64_t seed, uint64_t round, int32_t* idx_out,
+                             uint32_t* dev_err, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+SMCSD_API const char* sd_status_string(sd_status s);
+
+/* Library ABI version (major * 100 + minor). */
+SMCSD_API int sd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SMCSD_H_ */

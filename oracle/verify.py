@@ -25,7 +25,9 @@ not print the rule; this is the textbook speculative-sampling rule:
 Edge cases: a draft token outside [0, V) is rejected (accept probability 0)
 and raises the token error bit.  A non-finite target or draft row at a
 position the sequence reaches stops the sequence there: accepted_len is that
-position, no token is emitted at it, and the non-finite bit is raised.
+position, no token is emitted at it.  The non-finite bit is raised for any
+non-finite row among the K verified positions (its TV is NaN) and for the
+target row K+1 when the sequence reaches it.
 
 Parity status: the accept rule and residual are pinned by exhaustive
 enumeration at V = 4, K = 2 (the emitted token law equals the target law to
@@ -82,6 +84,8 @@ def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd):
         a, lse_t = row_log_softmax(zT[b], tau)
         d, lse_d = row_log_softmax(zD[b], tau)
         tv[b] = total_variation(a[:K], lse_t[:K], d, lse_d)
+        if np.isnan(lse_t[:K]).any() or np.isnan(lse_d).any():
+            err |= DEV_NONFINITE      # a NaN TV is reported even past the first rejection
         done = False
         for k in range(K):
             if np.isnan(lse_t[k]) or np.isnan(lse_d[k]):

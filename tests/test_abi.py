@@ -1,0 +1,80 @@
+"""The C-ABI library loads and exports every symbol include/smcsd.h declares (no GPU)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import resample_online_log_b200 as lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "smcsd.h")).read()
+    return sorted(set(re.findall(r"SMCSD_API\s+[\w\s\*]+?\b(\w+)\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    assert set(syms) == set(lib.EXPORTS), syms
+
+
+def test_library_exports_every_declared_symbol():
+    assert os.path.exists(lib.LIB_PATH), "build libsmcsd.so first (__graft_entry__.build())"
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for s in declared_symbols():
+        assert s in exported, s
+    L = lib.load()
+    for s in declared_symbols():
+        assert hasattr(L, s)
+
+
+def test_status_strings_and_version():
+    assert lib.status_string(lib.SD_OK) == "ok"
+    assert "invalid" in lib.status_string(lib.SD_ERR_INVALID_ARG)
+    assert lib.version() >= 100
+
+
+def test_host_argument_checks_need_no_gpu():
+    L = lib.load()
+    vp = ctypes.c_void_p
+    # N = 0 -> invalid before anything touches CUDA
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 0, 1, 10, 10, vp(1), 1.0, 0, 0, None, vp(1), vp(1),
+                         None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
+    # tau <= 0, ld < V
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 10, vp(1), 0.0, 0, 0, None, vp(1), vp(1),
+                         None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 9, vp(1), 1.0, 0, 0, None, vp(1), vp(1),
+                         None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
+    # B = 0 is an empty batch: OK, nothing enqueued
+    assert L.smcsd_score(None, None, 1, 0, 1, 1, 10, 10, None, 1.0, 0, 0, None, None, None,
+                         None, None, None, None, None, None) == lib.SD_OK
+    # missing required outputs
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 10, vp(1), 1.0, 0, 0, None, None, vp(1),
+                         None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
+    assert L.smcsd_resample(vp(1), 1, 0, 0, 0, None, None, vp(1), None, None) == lib.SD_ERR_INVALID_ARG
+    assert L.smcsd_resample(vp(1), 1, 9000, 0, 0, None, None, vp(1), None, None) == lib.SD_ERR_UNSUPPORTED
+    assert L.kv_pagetable_remap(vp(16), vp(16), 1, 1, 4, vp(16), vp(1), 2, None, None, 0, None,
+                                None) == lib.SD_ERR_INVALID_ARG     # tok_in without tok_out
+    assert L.kv_pagetable_remap(vp(16), vp(16), 1, 1, 4, vp(16), None, 0, None, None, 0, None,
+                                None) == lib.SD_ERR_INVALID_ARG     # aliasing pt_in / pt_out
+    assert L.sd_verify_reject(vp(1), vp(1), 1, 1, 0, 10, 10, vp(1), 1.0, 0, 0, vp(1), vp(1), None,
+                              None, None) == lib.SD_ERR_INVALID_ARG  # K = 0
+    assert L.gumbel_topk(vp(1), 1, 1, 10, 10, 11, 1.0, 0, 0, vp(1), None, None, None,
+                         None) == lib.SD_ERR_INVALID_ARG            # k > V
+    assert L.gumbel_topk_sparse(vp(1), vp(1), 1, 10, 11, 1.0, 0, 0, vp(1), None,
+                                None) == lib.SD_ERR_INVALID_ARG     # k > L
+
+
+def test_product_path_has_no_oracle_dependency():
+    pkg = os.path.join(ROOT, "resample_online_log_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f

@@ -1,0 +1,124 @@
+"""GPU parity of smcsd_resample and kv_pagetable_remap against the oracle, and of a
+whole SMC-SD round (score -> resample -> remap)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import resample_online_log_b200 as lib
+import synth
+from synth import gen
+from tests.parity import close, discrete, requires_gpu, to_dev
+
+pytestmark = [pytest.mark.gpu, requires_gpu]
+
+
+def run_resample(logw, seed, rnd):
+    B, N = logw.shape
+    lw = to_dev(np.asarray(logw, dtype=np.float64))
+    anc = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    W = torch.empty((B, N), dtype=torch.float64, device="cuda")
+    ess = torch.empty((B,), dtype=torch.float64, device="cuda")
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    lib.smcsd_resample(lw, seed, rnd, anc, w_out=W, ess_out=ess, dev_err=err)
+    torch.cuda.synchronize()
+    return dict(anc=anc.cpu().numpy(), W=W.cpu().numpy(), ess=ess.cpu().numpy(), err=int(err.item()))
+
+
+@pytest.mark.parametrize("B,N,scale", [(7, 1, 1.0), (64, 4, 2.0), (256, 32, 3.0), (3, 1000, 1.0),
+                                       (2, 8192, 5.0), (5, 33, 0.01)])
+def test_resample_parity(B, N, scale):
+    rng = np.random.default_rng(B * 1000 + N)
+    logw = rng.standard_normal((B, N)) * scale
+    g = run_resample(logw, seed=B, rnd=N)
+    o = oracle.smcsd_resample(logw, seed=B, rnd=N)
+    close(g["W"], o["W"], 1e-12, "W")
+    close(g["ess"], o["ess"], 1e-9 * N, "ess")
+    discrete(g["anc"], o["ancestors"], o["margin"], "ancestors")
+    assert g["err"] == 0
+    assert np.allclose(g["W"].sum(axis=1), 1.0, atol=1e-12)
+    counts = np.stack([np.bincount(a, minlength=N) for a in g["anc"]])
+    assert np.all(counts >= np.floor(N * g["W"]) - 1e-9) and np.all(counts <= np.ceil(N * g["W"]) + 1e-9)
+
+
+def test_resample_edge_cases():
+    logw = np.array([[0.0, np.nan, 1.0], [-np.inf, -np.inf, -np.inf], [0.0, 0.0, 0.0],
+                     [-np.inf, 3.0, -np.inf]])
+    g = run_resample(logw, 1, 0)
+    o = oracle.smcsd_resample(logw, 1, 0)
+    assert g["err"] == o["err"] == oracle.DEV_NONFINITE
+    assert np.array_equal(g["anc"], o["ancestors"])
+    assert np.all(g["anc"][3] == 1) and abs(g["ess"][3] - 1.0) < 1e-15
+    close(g["W"], o["W"], 1e-12, "W")
+
+
+def run_remap(pt, anc, num_pages=None, tok=None):
+    B, N, P = pt.shape
+    pti = to_dev(pt.astype(np.int32))
+    pto = torch.empty_like(pti)
+    an = to_dev(anc.astype(np.int32))
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    ref = None if num_pages is None else torch.empty((num_pages,), dtype=torch.int32, device="cuda")
+    ti = to = None
+    if tok is not None:
+        ti = to_dev(tok.astype(np.int32))
+        to = torch.empty_like(ti)
+    lib.kv_pagetable_remap(pti, an, pto, tok_in=ti, tok_out=to, page_refcnt=ref,
+                           num_pages=num_pages or 0, dev_err=err)
+    torch.cuda.synchronize()
+    return dict(pt=pto.cpu().numpy(), ref=None if ref is None else ref.cpu().numpy(),
+                tok=None if to is None else to.cpu().numpy(), err=int(err.item()))
+
+
+@pytest.mark.parametrize("B,N,P,T", [(1, 1, 1, 0), (4, 8, 128, 5), (3, 5, 7, 3), (256, 32, 128, 9)])
+def test_remap_parity(B, N, P, T):
+    rng = np.random.default_rng(B + N + P)
+    pt = gen.page_table(B, B, N, P)
+    pt[0, 0, -1] = -1
+    anc = np.sort(rng.integers(0, N, size=(B, N)), axis=1)
+    tok = rng.integers(0, 50000, size=(B, N, T)) if T else None
+    g = run_remap(pt, anc, num_pages=B * N * P, tok=tok)
+    o = oracle.kv_pagetable_remap(pt, anc, num_pages=B * N * P, tok_in=tok)
+    assert np.array_equal(g["pt"], o["pt_out"])
+    assert np.array_equal(g["ref"], o["refcnt"])
+    if T:
+        assert np.array_equal(g["tok"], o["tok_out"])
+    assert g["err"] == o["err"] == 0
+
+
+def test_remap_faults():
+    pt = gen.page_table(0, 2, 3, 6)
+    pt[1, 2, 4] = 10_000
+    anc = np.array([[0, 0, 3], [1, 2, 2]])
+    g = run_remap(pt, anc, num_pages=36)
+    o = oracle.kv_pagetable_remap(pt, anc, num_pages=36)
+    assert g["err"] == o["err"] == (oracle.DEV_PAGE_OOB | oracle.DEV_ANCESTOR_OOB)
+    assert np.array_equal(g["pt"], o["pt_out"]) and np.array_equal(g["ref"], o["refcnt"])
+
+
+def test_full_round_smc_small():
+    """score -> resample -> remap on the small SMC-SD config, each stage checked."""
+    cfg = synth.CONFIGS["smc_small"]
+    h = gen.gen_config_rows(cfg)
+    B, N, R, K = cfg.B, cfg.N, cfg.R, cfg.K
+    zT, zD = to_dev(h["zT"]), to_dev(h["zD"])
+    x = to_dev(h["draft"].astype(np.int32))
+    logw = torch.empty((B, N), dtype=torch.float64, device="cuda")
+    bonus = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    toks = torch.empty((B, N, R), dtype=torch.int32, device="cuda")
+    anc = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    pt = to_dev(gen.page_table(cfg.seed, B, N, cfg.P))
+    pt_out = torch.empty_like(pt)
+    tok_out = torch.empty_like(toks)
+    lib.smcsd_score(zT, zD, x, cfg.tau, cfg.seed, 3, logw, bonus, tokens_out=toks)
+    lib.smcsd_resample(logw, cfg.seed, 3, anc)
+    lib.kv_pagetable_remap(pt, anc, pt_out, tok_in=toks, tok_out=tok_out)
+    torch.cuda.synchronize()
+    o = oracle.smcsd_score(h["zT"], h["zD"], h["draft"], cfg.tau, cfg.seed, 3)
+    r = oracle.smcsd_resample(o["logw"], cfg.seed, 3)
+    discrete(bonus.cpu().numpy(), o["bonus"], o["bonus_margin"], "bonus")
+    discrete(anc.cpu().numpy(), r["ancestors"], r["margin"], "ancestors")
+    m = oracle.kv_pagetable_remap(pt.cpu().numpy(), r["ancestors"], tok_in=o["tokens"])
+    assert np.array_equal(pt_out.cpu().numpy(), m["pt_out"])
+    assert np.array_equal(tok_out.cpu().numpy(), m["tok_out"])

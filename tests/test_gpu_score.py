@@ -1,0 +1,206 @@
+"""GPU parity of smcsd_score against the oracle, through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import resample_online_log_b200 as lib
+import synth
+from synth import gen
+from tests.parity import TOL_LOGW, TOL_LSE, TOL_TV, bf16_dev, close, discrete, requires_gpu, to_dev
+
+pytestmark = [pytest.mark.gpu, requires_gpu]
+
+
+def run_score(zT, zD, x, tau, seed, rnd, dtype="bf16", logw_prev=None, ld=None):
+    B, N, R, V = zT.shape
+    K = R - 1
+    dev = "cuda"
+    if dtype == "bf16":
+        t, d = bf16_dev(zT), bf16_dev(zD)
+    else:
+        t, d = to_dev(zT.astype(np.float32)), to_dev(zD.astype(np.float32))
+    if ld is not None and ld != V:
+        tt = torch.zeros((B, N, R, ld), dtype=t.dtype, device=dev)
+        dd = torch.zeros((B, N, R, ld), dtype=t.dtype, device=dev)
+        tt[..., :V] = t
+        dd[..., :V] = d
+        t, d = tt[..., :V], dd[..., :V]
+    xs = to_dev(np.asarray(x, dtype=np.int32))
+    out = dict(
+        logw=torch.empty((B, N), dtype=torch.float64, device=dev),
+        bonus=torch.empty((B, N), dtype=torch.int32, device=dev),
+        tv=torch.empty((B, N, R), dtype=torch.float32, device=dev),
+        tokens=torch.empty((B, N, R), dtype=torch.int32, device=dev),
+        lse=torch.empty((B, N, R, 2), dtype=torch.float64, device=dev),
+        lp=torch.empty((B, N, K, 2), dtype=torch.float64, device=dev),
+        err=torch.zeros((1,), dtype=torch.int32, device=dev))
+    prev = None if logw_prev is None else to_dev(np.asarray(logw_prev, dtype=np.float64))
+    lib.smcsd_score(t, d, xs, tau, seed, rnd, out["logw"], out["bonus"], logw_prev=prev,
+                    tv_out=out["tv"], tokens_out=out["tokens"], lse_out=out["lse"],
+                    lp_out=out["lp"], dev_err=out["err"])
+    torch.cuda.synchronize()
+    res = {k: v.cpu().numpy() for k, v in out.items()}
+    res["err"] = int(res["err"][0])
+    return res
+
+
+def compare(g, o, name):
+    close(g["logw"], o["logw"], TOL_LOGW, name + ".logw")
+    close(g["tv"], o["tv"], TOL_TV, name + ".tv")
+    close(g["lse"], o["lse"], TOL_LSE, name + ".lse")
+    close(g["lp"], o["lp"], TOL_LSE, name + ".lp")
+    discrete(g["bonus"], o["bonus"], o["bonus_margin"], name + ".bonus")
+    K = o["tokens"].shape[-1] - 1
+    assert np.array_equal(g["tokens"][..., :K], o["tokens"][..., :K])
+    assert np.array_equal(g["tokens"][..., K], g["bonus"])
+    assert g["err"] == o["err"], (g["err"], o["err"])
+
+
+def rand_case(rng, B, N, K, V, scale=2.0, noise=1.0):
+    zT = (rng.standard_normal((B, N, K + 1, V)) * scale).astype(np.float32)
+    zD = (zT + rng.standard_normal(zT.shape) * noise).astype(np.float32)
+    zT = gen.bf16_bits_to_f32(gen.f32_to_bf16_bits(zT))
+    zD = gen.bf16_bits_to_f32(gen.f32_to_bf16_bits(zD))
+    x = rng.integers(0, V, size=(B, N, K)).astype(np.int32)
+    return zT, zD, x
+
+
+def test_smc_small_config_fp32():
+    cfg = synth.CONFIGS["smc_small"]
+    d = gen.gen_config_rows(cfg)
+    g = run_score(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed, 0, dtype="f32")
+    o = oracle.smcsd_score(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed, 0)
+    compare(g, o, "smc_small")
+
+
+@pytest.mark.parametrize("V,tau", [(1003, 0.8), (4096, 1.0), (33001, 0.7)])
+def test_ragged_vocab_bf16(V, tau):
+    rng = np.random.default_rng(V)
+    zT, zD, x = rand_case(rng, 2, 3, 2, V)
+    g = run_score(zT, zD, x, tau, 11, 5)
+    o = oracle.smcsd_score(zT, zD, x, tau, 11, 5)
+    compare(g, o, f"ragged{V}")
+
+
+def test_split_v_llama_vocab_bf16():
+    rng = np.random.default_rng(7)
+    zT, zD, x = rand_case(rng, 1, 3, 2, 128256, scale=3.0, noise=1.5)
+    g = run_score(zT, zD, x, 1.0, 3, 1)
+    o = oracle.smcsd_score(zT, zD, x, 1.0, 3, 1)
+    compare(g, o, "v128256")
+
+
+def test_fp32_multi_tile():
+    rng = np.random.default_rng(8)
+    zT, zD, x = rand_case(rng, 2, 2, 3, 40000)
+    g = run_score(zT, zD, x, 1.3, 4, 2, dtype="f32")
+    o = oracle.smcsd_score(zT, zD, x, 1.3, 4, 2)
+    compare(g, o, "f32_40000")
+
+
+def test_strided_unaligned_rows():
+    """ld*2 bytes is not a multiple of 16: the bulk-copy path is off, plain loads are used."""
+    rng = np.random.default_rng(9)
+    zT, zD, x = rand_case(rng, 2, 2, 2, 5000)
+    g = run_score(zT, zD, x, 0.9, 5, 0, ld=5003)
+    o = oracle.smcsd_score(zT, zD, x, 0.9, 5, 0)
+    compare(g, o, "strided")
+
+
+def test_padded_aligned_rows():
+    rng = np.random.default_rng(10)
+    zT, zD, x = rand_case(rng, 1, 4, 3, 32000)
+    g = run_score(zT, zD, x, 1.0, 6, 0, ld=32768)
+    o = oracle.smcsd_score(zT, zD, x, 1.0, 6, 0)
+    compare(g, o, "padded")
+
+
+def test_edge_cases_k0_n1_v1():
+    rng = np.random.default_rng(11)
+    zT, zD, x = rand_case(rng, 3, 2, 0, 700)          # K = 0: bonus only
+    g = run_score(zT, zD, x, 1.0, 1, 0)
+    o = oracle.smcsd_score(zT, zD, x, 1.0, 1, 0)
+    compare(g, o, "K0")
+    assert np.all(g["logw"] == 0.0)
+    zT, zD, x = rand_case(rng, 2, 1, 3, 900)          # N = 1
+    g = run_score(zT, zD, x, 1.0, 1, 0)
+    compare(g, oracle.smcsd_score(zT, zD, x, 1.0, 1, 0), "N1")
+    zT, zD, x = rand_case(rng, 2, 2, 2, 1)            # V = 1: point masses
+    g = run_score(zT, zD, x, 1.0, 1, 0)
+    compare(g, oracle.smcsd_score(zT, zD, x, 1.0, 1, 0), "V1")
+    assert np.all(g["bonus"] == 0) and np.all(g["tv"] == 0)
+
+
+def test_logw_prev_is_added():
+    rng = np.random.default_rng(12)
+    zT, zD, x = rand_case(rng, 2, 4, 2, 3000)
+    prev = rng.standard_normal((2, 4))
+    g = run_score(zT, zD, x, 1.0, 2, 9, logw_prev=prev)
+    compare(g, oracle.smcsd_score(zT, zD, x, 1.0, 2, 9, logw_prev=prev), "prev")
+
+
+def test_identical_rows_invariants():
+    rng = np.random.default_rng(13)
+    zT, _, x = rand_case(rng, 2, 4, 3, 128256)
+    g = run_score(zT, zT.copy(), x, 0.7, 3, 3)
+    assert np.all(g["logw"] == 0.0)
+    assert np.all(g["tv"] == 0.0)
+
+
+def test_faults_set_error_bits():
+    rng = np.random.default_rng(14)
+    zT, zD, x = rand_case(rng, 1, 3, 2, 2000)
+    x[0, 0, 1] = 2000                       # token out of range
+    zT[0, 1, 2, 17] = np.nan                # NaN in particle 1's bonus row
+    zD[0, 2, :, :] = -np.inf                # particle 2: all draft rows -inf
+    g = run_score(zT, zD, x, 1.0, 1, 0)
+    o = oracle.smcsd_score(zT, zD, x, 1.0, 1, 0)
+    assert g["err"] == o["err"] == (oracle.DEV_TOKEN_OOB | oracle.DEV_NONFINITE)
+    close(g["logw"], o["logw"], TOL_LOGW, "faults.logw")
+    close(g["tv"], o["tv"], TOL_TV, "faults.tv")
+    assert g["bonus"][0, 1] == -1 and o["bonus"][0, 1] == -1
+    discrete(g["bonus"], o["bonus"], o["bonus_margin"], "faults.bonus")
+
+
+def test_reruns_bit_identical():
+    rng = np.random.default_rng(15)
+    zT, zD, x = rand_case(rng, 2, 8, 4, 128256)
+    a = run_score(zT, zD, x, 1.0, 77, 4)
+    b = run_score(zT, zD, x, 1.0, 77, 4)
+    for key in ("logw", "tv", "bonus", "lse", "lp", "tokens"):
+        assert np.array_equal(a[key], b[key], equal_nan=True), key
+
+
+@pytest.mark.parametrize("name,seqs", [("smc_batch", [0, 37]), ("smc_scale", [5, 200])])
+def test_full_size_config_sampled(name, seqs):
+    """Whole config on the GPU (inputs built on the device), sampled sequences checked
+    against the oracle on host-built inputs; the device bytes of those sequences must
+    equal the host generator's."""
+    from synth import device as sdev
+    cfg = synth.CONFIGS[name]
+    d = sdev.gen_config_device(cfg)
+    B, N, R, V, K = cfg.B, cfg.N, cfg.R, cfg.V, cfg.K
+    out_logw = torch.empty((B, N), dtype=torch.float64, device="cuda")
+    out_bonus = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    out_tv = torch.empty((B, N, R), dtype=torch.float32, device="cuda")
+    out_lp = torch.empty((B, N, K, 2), dtype=torch.float64, device="cuda")
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    lib.smcsd_score(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed, 1, out_logw, out_bonus,
+                    tv_out=out_tv, lp_out=out_lp, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for b in seqs:
+        h = gen.gen_config_rows(cfg, seqs=[b])
+        dev_t = d["zT"][b].float().cpu().numpy()
+        dev_d = d["zD"][b].float().cpu().numpy()
+        assert np.array_equal(dev_t, h["zT"][0]) and np.array_equal(dev_d, h["zD"][0])
+        assert np.array_equal(d["draft"][b].cpu().numpy(), h["draft"][0])
+        o = oracle.smcsd_score(h["zT"], h["zD"], h["draft"], cfg.tau, cfg.seed, 1)
+        close(out_logw[b:b + 1].cpu().numpy(), o["logw"], TOL_LOGW, f"{name}[{b}].logw")
+        close(out_tv[b:b + 1].cpu().numpy(), o["tv"], TOL_TV, f"{name}[{b}].tv")
+        close(out_lp[b:b + 1].cpu().numpy(), o["lp"], TOL_LSE, f"{name}[{b}].lp")
+        discrete(out_bonus[b:b + 1].cpu().numpy(), o["bonus"], o["bonus_margin"], f"{name}[{b}].bonus")
+    del d
+    torch.cuda.empty_cache()

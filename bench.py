@@ -189,6 +189,8 @@ def run_ours(args, rank, world, local):
     from synth import gen
 
     cfg = gen.CONFIGS[WORKLOAD]
+    if args.sequences:  # a smaller case of the same workload (profiling)
+        cfg = gen.SynthConfig(**{**cfg.__dict__, "B": args.sequences})
     if rank:  # disjoint synthetic sequences per replica
         cfg = gen.SynthConfig(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
     B, N, R, K, V, P = cfg.B, cfg.N, cfg.R, cfg.K, cfg.V, cfg.P
@@ -259,7 +261,8 @@ def run_ours(args, rank, world, local):
         "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": B, "N": N, "K": K, "V": V, "logits": cfg.dtype,
+        "config": {"workload": WORKLOAD if not args.sequences else f"{WORKLOAD}[B={B}]",
+                   "B": B, "N": N, "K": K, "V": V, "logits": cfg.dtype,
                    "tau": cfg.tau, "pages_per_particle": P, "parallelism": f"replicas{world}",
                    "l2": "inputs (37.8 GB) larger than L2; no flush"},
         "hbm_TBps_score": achieved / 1e3,
@@ -320,6 +323,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sequences", type=int, default=0,
+                    help="run B sequences of the workload instead of all 256 (profiling)")
     args = ap.parse_args()
     rank, world, local = dist_init()
     try:

@@ -48,10 +48,10 @@ def resample_offset(seed, rnd, b):
     return float(uniform_from_bits(row_scalar_word(seed, rnd, STREAM_RESAMPLE, b)))
 
 
-def smcsd_resample(logw, seed, rnd):
+def smcsd_resample(logw, seed, rnd, b0=0):
     """Normalise log-weights, compute ESS and draw systematic ancestors.
 
-    logw: [B, N].  Returns dict(W [B,N], ess [B], ancestors [B,N], margin [B,N], err).
+    logw: [B, N]; b0 = global index of the first sequence (Philox row id).  Returns dict(W [B,N], ess [B], ancestors [B,N], margin [B,N], err).
     A sequence whose log-weights hold NaN or +inf, or are all -inf, gets NaN
     weights and ESS, identity ancestors, and raises the non-finite error bit.
     """
@@ -74,5 +74,5 @@ def smcsd_resample(logw, seed, rnd):
         w = np.exp(lw - m)
         W[b] = w / w.sum()
         ess[b] = 1.0 / np.sum(W[b] ** 2)
-        anc[b], margin[b] = systematic_ancestors(W[b], resample_offset(seed, rnd, b))
+        anc[b], margin[b] = systematic_ancestors(W[b], resample_offset(seed, rnd, b0 + b))
     return dict(W=W, ess=ess, ancestors=anc, margin=margin, err=err)

@@ -86,12 +86,14 @@ def bonus_noise(seed, rnd, row_id, V):
     return gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_BONUS, row_id, V)))
 
 
-def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None):
+def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None, b0=0):
     """Score one SMC-SD round for B sequences x N particles x (K+1) positions.
 
     zT, zD: [B, N, K+1, V] target / draft logits (any float dtype; widened to fp64).
     draft_tokens: [B, N, K] int, token x_{k+1} scored at row k.
     logw_prev: optional [B, N] fp64 log-weights carried from the last round.
+    b0: global index of the first sequence when these B sequences are a sample
+        of a larger batch (Philox row ids use the global particle index).
 
     Returns a dict with
       lse    [B, N, K+1, 2]  (lse of target row, lse of draft row)
@@ -139,7 +141,7 @@ def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None):
             logw[b, n] = acc
             tokens[b, n, :K] = draft_tokens[b, n]
             if not np.isnan(lse_t[K]):
-                g = bonus_noise(seed, rnd, b * N + n, V)
+                g = bonus_noise(seed, rnd, (b0 + b) * N + n, V)
                 idx, mg = gumbel_argmax(a[K] + g)
                 bonus[b, n] = idx
                 margin[b, n] = mg

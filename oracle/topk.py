@@ -45,8 +45,9 @@ def _ordered_topk(score, k):
     return sel, margin
 
 
-def gumbel_topk(z, k, tau, seed, rnd):
-    """Dense rows z [rows, V] -> dict(idx [rows,k], score [rows,k], logp [rows,k], margin [rows], err)."""
+def gumbel_topk(z, k, tau, seed, rnd, r0=0):
+    """Dense rows z [rows, V] -> dict(idx [rows,k], score [rows,k], logp [rows,k], margin [rows], err).
+    r0 = global index of the first row (Philox row id)."""
     z = np.asarray(z)
     rows, V = z.shape
     idx = np.full((rows, k), -1, dtype=np.int64)
@@ -60,7 +61,7 @@ def gumbel_topk(z, k, tau, seed, rnd):
         if bad[r]:
             err |= DEV_NONFINITE
             continue
-        g = gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_TOPK_DENSE, r, V)))
+        g = gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_TOPK_DENSE, r0 + r, V)))
         sc = s_all[r] + g
         sel, margin[r] = _ordered_topk(sc, k)
         idx[r] = sel
@@ -70,7 +71,7 @@ def gumbel_topk(z, k, tau, seed, rnd):
     return dict(idx=idx, score=score, logp=logp, margin=margin, err=err)
 
 
-def gumbel_topk_sparse(idx_in, prob, k, tau, seed, rnd):
+def gumbel_topk_sparse(idx_in, prob, k, tau, seed, rnd, r0=0):
     """Sparse rows (idx [rows, L], prob [rows, L]) -> dict(idx [rows,k], margin [rows], err)."""
     idx_in = np.asarray(idx_in, dtype=np.int64)
     prob = np.asarray(prob, dtype=np.float64)
@@ -86,7 +87,7 @@ def gumbel_topk_sparse(idx_in, prob, k, tau, seed, rnd):
             continue
         with np.errstate(divide="ignore"):
             s = np.where(pr > 0, np.log(np.where(pr > 0, pr, 1.0)) / t, -np.inf)
-        g = gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_TOPK_SPARSE, r, L)))
+        g = gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_TOPK_SPARSE, r0 + r, L)))
         sel, margin[r] = _ordered_topk(s + g, k)
         out[r] = np.where(sel >= 0, idx_in[r, np.maximum(sel, 0)], -1)
     return dict(idx=out, margin=margin, err=err)

@@ -60,10 +60,11 @@ def accept_uniform(seed, rnd, row_id):
     return float(uniform_from_bits(row_scalar_word(seed, rnd, STREAM_ACCEPT, row_id)))
 
 
-def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd):
+def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd, b0=0):
     """Verify K drafted tokens per sequence.
 
-    zT: [B, K+1, V], zD: [B, K, V], draft_tokens: [B, K].
+    zT: [B, K+1, V], zD: [B, K, V], draft_tokens: [B, K]; b0 = global index of
+    the first sequence (Philox row ids use the global sequence index).
     Returns dict(accepted_len [B], out_tokens [B, K+1], tv [B, K],
                  accept_margin [B, K] (inf where no decision was taken),
                  token_margin [B], err).
@@ -96,7 +97,7 @@ def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd):
             p = np.exp(a[k] - lse_t[k])
             q = np.exp(d[k] - lse_d[k])
             x = int(draft[b, k])
-            u = accept_uniform(seed, rnd, b * R + k)
+            u = accept_uniform(seed, rnd, (b0 + b) * R + k)
             if 0 <= x < V:
                 accept = u * q[x] < p[x]
                 acc_margin[b, k] = abs(u - accept_probability(p, q, x))
@@ -107,7 +108,7 @@ def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd):
                 out[b, k] = x
                 continue
             g = gumbel_from_uniform(uniform_from_bits(
-                stream_words(seed, rnd, STREAM_RESIDUAL, b * R + k, V)))
+                stream_words(seed, rnd, STREAM_RESIDUAL, (b0 + b) * R + k, V)))
             r = np.maximum(p - q, 0.0)
             if (r > 0).any():
                 with np.errstate(divide="ignore"):
@@ -127,7 +128,7 @@ def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd):
         if np.isnan(lse_t[K]):
             err |= DEV_NONFINITE
             continue
-        g = gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_BONUS, b, V)))
+        g = gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_BONUS, b0 + b, V)))
         tok, mg = gumbel_argmax(a[K] + g)
         out[b, K] = tok
         tok_margin[b] = mg

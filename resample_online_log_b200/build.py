@@ -29,8 +29,10 @@ def build(verbose=False, jobs=None):
     for p in procs:
         if p.wait() != 0:
             raise RuntimeError("nvcc failed")
-    cmd = ["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", LIB, *objs,
-           "-lcudart"]
+    # Static CUDA runtime with its symbols kept local: the library carries its own
+    # runtime and never binds to another copy already loaded in the process.
+    cmd = ["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "--cudart", "static",
+           "-Xlinker", "--exclude-libs,ALL", "-o", LIB, *objs]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -7,9 +7,7 @@
 // systematic resampling, run every round:
 //   W_j = exp(logw_j - max) / sum,  ESS = 1 / sum W_j^2,
 //   C_j = W_0 + ... + W_j,  U_i = (i + u0) / N,  a_i = min{ j : C_j > U_i }.
-// Each thread owns a contiguous run of particles, so the running sum is a
-// per-thread serial scan plus one block-wide scan of the run totals; the order
-// of every reduction is fixed, so results are bit-reproducible.
+// The order of every reduction is fixed, so results are bit-reproducible.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -80,21 +78,25 @@ __device__ double block_exclusive_scan_d(double v, double* scratch) {
   return scratch[warp] + (inc - v);
 }
 
+// Thread t owns particles t, t + T, t + 2T, ... so no thread ever touches two
+// adjacent doubles (every shared / global access is a naturally aligned
+// scalar).  The running sum is a block-wide scan over chunks of T particles
+// with a carried offset.  Shared layout: [0, 40) reduction scratch, then the
+// N weights / running sums, both 16-byte aligned.
 __global__ void resample_kernel(const double* __restrict__ logw, int N, uint64_t seed,
                                 uint64_t round, double* __restrict__ w_out,
                                 double* __restrict__ ess_out, int32_t* __restrict__ anc_out,
                                 uint32_t* dev_err) {
-  extern __shared__ double sh[];  // [0, N): weights then running sums; [N, N+33): scratch
-  double* scratch = sh + N;
+  extern __shared__ __align__(16) double sh_all[];
+  double* scratch = sh_all;
+  double* sh = sh_all + 40;
   const int b = blockIdx.x;
-  const int T = blockDim.x;
-  const int per = (N + T - 1) / T;
-  const int j0 = min(N, (int)threadIdx.x * per), j1 = min(N, j0 + per);
+  const int T = blockDim.x, t = threadIdx.x;
   const double* lw = logw + (int64_t)b * N;
 
   double m = -INFINITY;
   double badv = 0.0;
-  for (int j = j0; j < j1; ++j) {
+  for (int j = t; j < N; j += T) {
     const double v = lw[j];
     if (isnan(v) || v == INFINITY) badv = 1.0;
     m = fmax(m, v);
@@ -102,39 +104,46 @@ __global__ void resample_kernel(const double* __restrict__ logw, int N, uint64_t
   m = block_max_d(m, scratch);
   badv = block_max_d(badv, scratch);
   if (badv > 0.0 || m == -INFINITY) {
-    for (int j = j0; j < j1; ++j) {
+    for (int j = t; j < N; j += T) {
       if (w_out) w_out[(int64_t)b * N + j] = NAN;
       anc_out[(int64_t)b * N + j] = j;
     }
-    if (threadIdx.x == 0) {
+    if (t == 0) {
       if (ess_out) ess_out[b] = NAN;
       raise_err(dev_err, SD_DEV_NONFINITE);
     }
     return;
   }
   double s = 0.0;
-  for (int j = j0; j < j1; ++j) {
+  for (int j = t; j < N; j += T) {
     const double w = exp(lw[j] - m);
     sh[j] = w;
     s += w;
   }
   const double S = block_sum_d(s, scratch);
-  double sq = 0.0, run = 0.0;
-  for (int j = j0; j < j1; ++j) {
+  double sq = 0.0;
+  for (int j = t; j < N; j += T) {
     const double W = sh[j] / S;
+    sh[j] = W;
     if (w_out) w_out[(int64_t)b * N + j] = W;
     sq += W * W;
-    run += W;
-    sh[j] = run;  // local inclusive running sum
   }
   const double sumsq = block_sum_d(sq, scratch);
-  const double off = block_exclusive_scan_d(run, scratch);
-  for (int j = j0; j < j1; ++j) sh[j] += off;
+  // running sums C_j, chunk by chunk
+  double carry = 0.0;
+  for (int c0 = 0; c0 < N; c0 += T) {
+    const int j = c0 + t;
+    const double v = j < N ? sh[j] : 0.0;
+    const double ex = block_exclusive_scan_d(v, scratch);
+    const double total = block_sum_d(v, scratch);
+    if (j < N) sh[j] = carry + ex + v;
+    carry += total;
+  }
   __syncthreads();
-  if (threadIdx.x == 0 && ess_out) ess_out[b] = 1.0 / sumsq;
+  if (t == 0 && ess_out) ess_out[b] = 1.0 / sumsq;
   const Stream st(seed, round, SD_STREAM_RESAMPLE);
   const double u0 = uniform_f64(st.at(0, (uint32_t)b).x);
-  for (int i = j0; i < j1; ++i) {
+  for (int i = t; i < N; i += T) {
     const double U = ((double)i + u0) / (double)N;
     int lo = 0, hi = N;  // first j with C_j > U
     while (lo < hi) {
@@ -157,10 +166,9 @@ extern "C" sd_status smcsd_resample(const double* logw, int B, int N, uint64_t s
   if (N > kResampleMaxN) return SD_ERR_UNSUPPORTED;
   if (B == 0) return SD_OK;
   if (!logw || !ancestors_out) return SD_ERR_INVALID_ARG;
-  int threads = ((N + 7) / 8 + 31) / 32 * 32;  // about 8 particles per thread
+  int threads = (N + 31) / 32 * 32;  // one particle per thread up to 1024
   if (threads > 1024) threads = 1024;
-  if (threads < 32) threads = 32;
-  const size_t smem = (size_t)(N + 33) * sizeof(double);
+  const size_t smem = (size_t)(N + 40) * sizeof(double);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(resample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   resample_kernel<<<B, threads, smem, (cudaStream_t)stream>>>(logw, N, seed, round, w_out, ess_out,

@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     if (want_tv) {
       float tv = 0.f;
 #pragma unroll
-      for (int i = 0; i < EPT; ++i) tv += fabsf(xt[i] * scT - xd[i] * scD);
+      for (int i = 0; i < EPT; ++i) tv += fabsf(__fmul_rn(xt[i], scT) - __fmul_rn(xd[i], scD));
       tv = warp_sum(tv);
       if (lane == 0) st_peer_f32(peer_addr(&tl->tvp[par][rank][warp], 0), tv);
     }

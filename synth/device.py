@@ -21,7 +21,8 @@ def build(verbose=False):
     src = os.path.join(_HERE, "csrc", "synth.cu")
     out = os.path.join(_HERE, "libsynth.so")
     cmd = ["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
-           "-Xcompiler", "-fPIC", "-shared", "-o", out, src]
+           "-Xcompiler", "-fPIC", "-shared", "--cudart", "static", "-Xlinker", "--exclude-libs,ALL",
+           "-o", out, src]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -62,5 +62,7 @@ def bf16_dev(a_f32, device="cuda"):
     """Host fp32 array holding bf16-exact values -> device bf16 tensor (exact)."""
     t = torch.from_numpy(np.ascontiguousarray(a_f32, dtype=np.float32))
     bt = t.to(torch.bfloat16)
-    assert torch.equal(bt.to(torch.float32), t), "values are not bf16-exact"
+    back = bt.to(torch.float32)
+    same = (back == t) | (torch.isnan(back) & torch.isnan(t))
+    assert bool(same.all()), "values are not bf16-exact"
     return bt.to(device)

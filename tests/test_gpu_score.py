@@ -197,7 +197,7 @@ def test_full_size_config_sampled(name, seqs):
         dev_d = d["zD"][b].float().cpu().numpy()
         assert np.array_equal(dev_t, h["zT"][0]) and np.array_equal(dev_d, h["zD"][0])
         assert np.array_equal(d["draft"][b].cpu().numpy(), h["draft"][0])
-        o = oracle.smcsd_score(h["zT"], h["zD"], h["draft"], cfg.tau, cfg.seed, 1)
+        o = oracle.smcsd_score(h["zT"], h["zD"], h["draft"], cfg.tau, cfg.seed, 1, b0=b)
         close(out_logw[b:b + 1].cpu().numpy(), o["logw"], TOL_LOGW, f"{name}[{b}].logw")
         close(out_tv[b:b + 1].cpu().numpy(), o["tv"], TOL_TV, f"{name}[{b}].tv")
         close(out_lp[b:b + 1].cpu().numpy(), o["lp"], TOL_LSE, f"{name}[{b}].lp")

@@ -64,10 +64,10 @@ def test_verify_random(V, K, tau, noise):
     zT = gen.bf16_bits_to_f32(gen.f32_to_bf16_bits(zT))
     zD = gen.bf16_bits_to_f32(gen.f32_to_bf16_bits(zD))
     # draft tokens from q (host sampler of the test; any valid ids would do)
-    q = np.exp(zD - zD.max(axis=-1, keepdims=True))
+    zd64 = zD.astype(np.float64) / tau
+    q = np.exp(zd64 - zd64.max(axis=-1, keepdims=True))
     q /= q.sum(axis=-1, keepdims=True)
-    x = np.array([[rng.choice(V, p=q[b, k].astype(np.float64) / q[b, k].sum()) for k in range(K)]
-                  for b in range(B)], dtype=np.int32)
+    x = np.array([[rng.choice(V, p=q[b, k]) for k in range(K)] for b in range(B)], dtype=np.int32)
     g = run_verify(zT, zD, x, tau, 3, V)
     o = oracle.sd_verify_reject(zT, zD, x, tau, 3, V)
     compare(g, o, f"verify{V}")

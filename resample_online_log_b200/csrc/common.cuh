@@ -206,6 +206,30 @@ __device__ __forceinline__ void st_peer_f32(uint32_t a, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
 
+// Asynchronous store into a peer CTA's shared memory that completes `bytes`
+// of transaction count on the peer's mbarrier (both addresses from peer_addr).
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, float a, float b, float c, float d,
+                                            uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(raddr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t raddr, uint32_t v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                   raddr),
+               "r"(v), "r"(rbar)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+// Barrier among the first `n` threads of the CTA (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void bar_sync_n(int n) {
+  asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory");
+}
+
 __device__ __forceinline__ void raise_err(uint32_t* dev_err, uint32_t bits) {
   if (dev_err) atomicOr(dev_err, bits);
 }

@@ -70,11 +70,6 @@ struct ScoreArgs {
   uint32_t* dev_err;
 };
 
-struct XSlot {  // one CTA's per-row partials
-  float mT, sT, mD, sD;
-  float zxT, zxD, pad0, pad1;
-};
-
 struct Cand {  // screening partial: best point score, its bounds, best bound of the rest
   float s, lo, hi, ohi;
   int idx, pad0, pad1, pad2;
@@ -85,17 +80,42 @@ struct Cand64 {
   int idx, pad;
 };
 
-struct Tail {
-  uint64_t full[8];
-  XSlot xs[2];
+// One CTA's message for one row, pushed into every CTA of the cluster.
+struct alignas(16) Msg {
+  float mT, sT, mD, sD;  // (max, sum of exps relative to it) over its slice of each row
+  float zxT, zxD;        // raw logits of the draft token (owner CTA only)
+  float tvprev;          // this CTA's TV partial of its previous row
+  int aux;               // argmax entry of its target slice (rows that draw a token)
+};
+
+constexpr int kLogN = 4;
+// Row record handed from the leader's compute warps to its bookkeeping warp.
+struct alignas(16) LogEntry {
+  Msg m[kMaxCluster];
+  int64_t unit;
+  int k, x;
+};
+
+struct alignas(128) Tail {
+  uint64_t full[4];           // ring stages (bulk copies)
+  uint64_t rbar[2];           // row messages, by row parity
+  uint64_t cbar[2], dbar[2];  // candidate / fp64 messages, by use parity
+  uint64_t fbar, pad_bar;
+  uint64_t logfull[kLogN], logempty[kLogN];
+  Msg recv[2][kMaxCluster];
+  Cand crecv[2][kMaxCluster];
+  Cand64 drecv[2][kMaxCluster];
+  float frecv[kMaxCluster];
   float4 wpart[kMaxWarps];
-  float tvp[2][kMaxCluster][kMaxWarps];
+  float tvw[kMaxWarps];
+  float wargv[kMaxWarps];
+  int wargi[kMaxWarps];
   Cand wcand[kMaxWarps];
-  Cand xc;
   Cand64 wc64[kMaxWarps];
-  Cand64 xc64;
+  float zx[2][2];
   double lse64[2];
   int flag[4];
+  LogEntry log[kLogN];
 };
 
 __device__ __forceinline__ Cand cand_empty() {
@@ -459,6 +479,112 @@ __device__ __noinline__ int accept_test(double zxT, double zxD, double lseT, dou
 }
 
 // ------------------------------------------------------------------ the kernel
+// Message exchange: after its CTA-level reduction a CTA pushes one 32-byte Msg
+// into slot [rank] of every CTA of the cluster with st.async, which completes
+// transaction bytes on the receiver's mbarrier; each CTA arms its own barrier
+// for C messages and waits on it.  No cluster-wide barrier and no fence sits
+// on the per-row path.  Slots and barriers alternate by row parity: a CTA can
+// only send row r+2 after it has every row r+1 message, and every CTA reads
+// its row r slots before sending row r+1, so a slot is never overwritten
+// before it is read.
+
+__device__ __forceinline__ void send_row_msg(Tail* tl, int par, uint32_t rank, uint32_t C, int lane,
+                                             const Msg& m) {
+  if (lane < (int)C) {
+    const uint32_t ra = peer_addr(&tl->recv[par][rank], (uint32_t)lane);
+    const uint32_t rb = peer_addr(&tl->rbar[par], (uint32_t)lane);
+    st_async_v4(ra, m.mT, m.sT, m.mD, m.sD, rb);
+    st_async_v4(ra + 16, m.zxT, m.zxD, m.tvprev, __int_as_float(m.aux), rb);
+  }
+}
+
+// Bookkeeping warp of the leader CTA: fp64 lse, log-probs, log-weights, TV and
+// per-particle outputs, fed row by row through a small shared-memory ring so
+// that none of this sits on the compute warps' critical path.
+template <bool VERIFY>
+__device__ void bookkeep(const ScoreArgs& a, Tail* tl, uint32_t C, uint32_t cid, uint32_t G,
+                         int64_t nrows, bool want_tv) {
+  const int lane = threadIdx.x & 31;
+  double logw_acc = 0.0;
+  bool unit_bad = false;
+  int64_t prev_tv_idx = -1;
+  bool prev_bad = false;
+  const int64_t entries = nrows + ((want_tv && nrows > 0) ? 1 : 0);
+  for (int64_t it = 0; it < entries; ++it) {
+    const int slot = (int)(it % kLogN);
+    if (!mbar_wait(&tl->logfull[slot], (uint32_t)((it / kLogN) & 1)))
+      raise_err(a.dev_err, SD_DEV_TIMEOUT);
+    const LogEntry& e = tl->log[slot];
+    if (prev_tv_idx >= 0) {  // every message carries its CTA's TV partial of the previous row
+      float v = lane < (int)C ? e.m[lane].tvprev : 0.f;
+      v = warp_sum(v);
+      if (lane == 0) a.tv_out[prev_tv_idx] = prev_bad ? NAN : 0.5f * v;
+    }
+    if (it == nrows) {  // final record: only the last row's TV
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->logempty[slot]);
+      break;
+    }
+    const int64_t unit = e.unit;
+    const int k = e.k, x = e.x;
+    const bool hasD = !VERIFY || k < a.K;
+    const float pm1 = lane < (int)C ? e.m[lane].mT : -INFINITY;
+    const float ps1 = lane < (int)C ? e.m[lane].sT : 0.f;
+    const float pm2 = lane < (int)C ? e.m[lane].mD : -INFINITY;
+    const float ps2 = lane < (int)C ? e.m[lane].sD : 0.f;
+    const float MT = warp_max(pm1);
+    const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
+    const float MD = hasD ? warp_max(pm2) : 0.f;
+    const float SD = hasD ? warp_sum(part_term(pm2, ps2, MD, a.cT)) : 1.f;
+    const bool badT = !(MT > -INFINITY && MT < INFINITY && ST > 0.f && ST < INFINITY);
+    const bool badD = hasD && !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
+    const bool bad = badT || badD;
+    const int64_t rowT = unit * a.R + k;
+    const int64_t rowD = VERIFY ? unit * a.K + k : rowT;
+    if (!VERIFY) {
+      if (k == 0) {
+        logw_acc = 0.0;
+        unit_bad = false;
+      }
+      const double lse64T = row_lse64(pm1, ps1, MT, lane < (int)C, a.tau64);
+      const double lse64D = row_lse64(pm2, ps2, MD, lane < (int)C, a.tau64);
+      if (lane == 0) {
+        if (bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
+        if (a.lse_out) {
+          a.lse_out[rowT * 2 + 0] = badT ? NAN : lse64T;
+          a.lse_out[rowT * 2 + 1] = badD ? NAN : lse64D;
+        }
+        if (k < a.K) {
+          const bool x_ok = x >= 0 && x < a.V;
+          double lp = NAN, lq = NAN;
+          if (!x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
+          if (x_ok && !bad) {
+            const Msg& o = e.m[x / a.slice];
+            lp = (double)o.zxT / a.tau64 - lse64T;
+            lq = (double)o.zxD / a.tau64 - lse64D;
+          } else {
+            unit_bad = true;
+          }
+          logw_acc += lp - lq;
+          if (a.lp_out) {
+            a.lp_out[(unit * a.K + k) * 2 + 0] = lp;
+            a.lp_out[(unit * a.K + k) * 2 + 1] = lq;
+          }
+        } else {
+          const double prev = a.logw_prev ? a.logw_prev[unit] : 0.0;
+          a.logw_out[unit] = unit_bad ? NAN : prev + logw_acc;
+          if (a.tokens_out)
+            for (int j = 0; j < a.K; ++j) a.tokens_out[unit * a.R + j] = a.draft[unit * a.K + j];
+        }
+      }
+    }
+    prev_tv_idx = (want_tv && hasD) ? (VERIFY ? rowD : rowT) : -1;
+    prev_bad = bad;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tl->logempty[slot]);
+  }
+}
+
 template <typename TIn, int CPT, bool VERIFY>
 __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a) {
   constexpr int EPC = 16 / (int)sizeof(TIn);
@@ -467,7 +593,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nthr = blockDim.x, nwarps = nthr >> 5;
+  const int ncomp = blockDim.x - 32, nwarps = ncomp >> 5;  // last warp: bookkeeping
   const uint32_t rank = cluster_rank(), C = cluster_size();
   const uint32_t cid = cluster_id(), G = num_clusters();
   Tail* tl = reinterpret_cast<Tail*>(smem + (size_t)a.stages * 2 * a.stage_bytes);
@@ -479,13 +605,30 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
   const int64_t my_units = (int64_t)cid < a.units ? (a.units - 1 - cid) / G + 1 : 0;
   const int64_t nrows = my_units * a.R;
   const bool leader = rank == 0;
+  const bool want_tv = a.tv_out != nullptr;
 
   if (tid == 0) {
     for (int s = 0; s < a.stages; ++s) mbar_init(&tl->full[s], 1);
+    for (int p = 0; p < 2; ++p) {
+      mbar_init(&tl->rbar[p], 1);
+      mbar_init(&tl->cbar[p], 1);
+      mbar_init(&tl->dbar[p], 1);
+    }
+    mbar_init(&tl->fbar, 1);
+    for (int i = 0; i < kLogN; ++i) {
+      mbar_init(&tl->logfull[i], 1);
+      mbar_init(&tl->logempty[i], 1);
+    }
     fence_mbar_init();
   }
   __syncthreads();
-  cluster_sync();
+  cluster_sync();  // every CTA's barriers exist before anyone sends to them
+
+  if (warp == nwarps) {
+    if (leader) bookkeep<VERIFY>(a, tl, C, cid, G, nrows, want_tv);
+    cluster_sync();
+    return;
+  }
 
   const uint64_t pol = policy_evict_first();
   auto issue = [&](int64_t it) {
@@ -507,15 +650,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
   if (tid == 0)
     for (int64_t it = 0; it < nrows && it < a.stages; ++it) issue(it);
 
-  // Per-unit state.  Decisions are computed identically in every CTA of the
-  // cluster, so control flow (and the number of cluster barriers) matches.
-  double logw_acc = 0.0;  // leader, warp 0
-  bool unit_bad = false;  // leader, warp 0: some lp / lq invalid
-  bool done = false;      // verify: sequence finished
-  int acc_len = 0;        // verify
-  int emitted = -1;       // verify: the drawn token
-  int64_t prev_tv_idx = -1;
-  bool prev_bad = false;
+  bool done = false;  // verify: sequence finished (identical in every CTA)
+  int acc_len = 0;
+  int emitted = -1;
+  int uses = 0;       // candidate exchanges so far
+  int duses = 0;      // fp64 exchanges so far
+  int x_pref = (nrows > 0 && a.K > 0) ? a.draft[(int64_t)cid * a.K] : -1;
 
   float xt[EPT], xd[EPT];
 
@@ -528,35 +668,51 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     const bool hasD = !VERIFY || k < a.K;
     const int64_t rowT = unit * a.R + k;
     const int64_t rowD = VERIFY ? unit * a.K + k : rowT;
+    const bool draws = (k == a.K) || VERIFY;  // rows that may draw a token need the argmax
     if (k == 0) {
-      logw_acc = 0.0;
-      unit_bad = false;
       done = false;
       acc_len = 0;
       emitted = -1;
     }
-    const int x = k < a.K ? a.draft[unit * a.K + k] : -1;
+    const int x = k < a.K ? x_pref : -1;
     const bool x_ok = k < a.K && x >= 0 && x < a.V;
+    if (it + 1 < nrows) {  // prefetch the next row's draft token
+      const int64_t un = cid + ((it + 1) / a.R) * G;
+      const int kn = (int)((it + 1) % a.R);
+      x_pref = kn < a.K ? a.draft[un * a.K + kn] : -1;
+    }
 
     if (!mbar_wait(&tl->full[s], ph)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
     const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)s * 2 * a.stage_bytes);
-    const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)s * 2 * a.stage_bytes + a.stage_bytes);
+    const TIn* stD =
+        reinterpret_cast<const TIn*>(smem + (size_t)s * 2 * a.stage_bytes + a.stage_bytes);
     const TIn* gT = (const TIn*)a.zT + rowT * a.ld + s0;
     const TIn* gD = (const TIn*)a.zD + rowD * a.ld + s0;
 
-    const float mt = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, tid, nthr);
+    const float mt = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, tid, ncomp);
     float md = -INFINITY;
-    if (hasD) md = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, tid, nthr);
-    // the owner of the draft token's entry records its raw logits
+    if (hasD) md = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, tid, ncomp);
+    int amax = 0x7FFFFFFF;  // this thread's first entry equal to its max (global index)
+    if (draws) {
+#pragma unroll
+      for (int i = EPT - 1; i >= 0; --i)
+        if (xt[i] == mt) amax = s0 + (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
+    }
     if (x_ok && x >= s0 && x < s0 + len) {
       const int le = x - s0;
-      if (((le / EPC) % nthr) == tid) {
-        tl->xs[par].zxT = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
-        tl->xs[par].zxD = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
+      if (((le / EPC) % ncomp) == tid) {
+        tl->zx[par][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
+        tl->zx[par][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
       }
     }
     const float mwT = warp_max(mt);
     const float mwD = hasD ? warp_max(md) : -INFINITY;
+    if (draws) {  // warp argmax: lowest index among lanes holding the warp max
+      int ai = (mt == mwT) ? amax : 0x7FFFFFFF;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ai = min(ai, __shfl_xor_sync(0xffffffffu, ai, o));
+      amax = ai;
+    }
     const float mwTs = mwT == -INFINITY ? 0.f : mwT;
     const float mwDs = mwD == -INFINITY ? 0.f : mwD;
     float sT = exp_slice<EPT>(xt, mwTs, a.cT);
@@ -564,32 +720,42 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     if (hasD) sD = exp_slice<EPT>(xd, mwDs, a.cT);
     sT = warp_sum(sT);
     if (hasD) sD = warp_sum(sD);
-    if (lane == 0) tl->wpart[warp] = make_float4(mwT, sT, mwD, sD);
-    __syncthreads();  // (A) the stage is now free; warp partials are visible
+    if (lane == 0) {
+      tl->wpart[warp] = make_float4(mwT, sT, mwD, sD);
+      tl->wargv[warp] = mwT;
+      tl->wargi[warp] = amax;
+    }
+    bar_sync_n(ncomp);  // (A) the stage is free; warp partials are visible
     if (tid == 0 && it + a.stages < nrows) issue(it + a.stages);
     if (warp == 0) {
-      const float4 wp = lane < nwarps ? tl->wpart[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-      const float M1 = warp_max(wp.x), M2 = warp_max(wp.z);
-      const float S1 = warp_sum(part_term(wp.x, wp.y, M1, a.cT));
-      const float S2 = warp_sum(part_term(wp.z, wp.w, M2, a.cT));
-      if (lane == 0) {
-        tl->xs[par].mT = M1;
-        tl->xs[par].sT = S1;
-        tl->xs[par].mD = M2;
-        tl->xs[par].sD = S2;
-      }
+      const float4 wp =
+          lane < nwarps ? tl->wpart[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+      Msg m;
+      m.mT = warp_max(wp.x);
+      m.mD = warp_max(wp.z);
+      m.sT = warp_sum(part_term(wp.x, wp.y, m.mT, a.cT));
+      m.sD = warp_sum(part_term(wp.z, wp.w, m.mD, a.cT));
+      float tvp = (lane < nwarps && it > 0) ? tl->tvw[lane] : 0.f;
+      m.tvprev = warp_sum(tvp);
+      int ai = 0x7FFFFFFF;
+      if (draws && lane < nwarps && tl->wargv[lane] == m.mT) ai = tl->wargi[lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ai = min(ai, __shfl_xor_sync(0xffffffffu, ai, o));
+      m.aux = ai;
+      const bool owner = x_ok && x >= s0 && x < s0 + len;
+      m.zxT = owner ? tl->zx[par][0] : 0.f;
+      m.zxD = owner ? tl->zx[par][1] : 0.f;
+      if (lane == 0) mbar_arrive_expect_tx(&tl->rbar[par], C * (uint32_t)sizeof(Msg));
+      send_row_msg(tl, par, rank, C, lane, m);
     }
-    cluster_sync();  // (B) all CTAs' partials of this row are visible
+    if (!mbar_wait(&tl->rbar[par], (uint32_t)((it >> 1) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
 
-    // Rebuild the row's normalisers from the C partials (every warp, same order).
-    float pm1 = -INFINITY, ps1 = 0.f, pm2 = -INFINITY, ps2 = 0.f;
-    if (lane < (int)C) {
-      const uint32_t pa = peer_addr(&tl->xs[par], lane);
-      pm1 = ld_peer_f32(pa + 0);
-      ps1 = ld_peer_f32(pa + 4);
-      pm2 = ld_peer_f32(pa + 8);
-      ps2 = ld_peer_f32(pa + 12);
-    }
+    // Rebuild the row's normalisers from the C messages (every warp, same order).
+    const Msg* rv = tl->recv[par];
+    const float pm1 = lane < (int)C ? rv[lane].mT : -INFINITY;
+    const float ps1 = lane < (int)C ? rv[lane].sT : 0.f;
+    const float pm2 = lane < (int)C ? rv[lane].mD : -INFINITY;
+    const float ps2 = lane < (int)C ? rv[lane].sD : 0.f;
     const float MT = warp_max(pm1);
     const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
     const float MD = hasD ? warp_max(pm2) : 0.f;
@@ -598,83 +764,53 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     const bool badD = hasD && !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
     const bool bad = badT || badD;
 
-    // fp64 lse of both rows (warp 0 of every CTA; lanes < C hold the partials)
-    double lse64T = 0.0, lse64D = 0.0, zxT = 0.0, zxD = 0.0;
-    if (warp == 0) {
-      lse64T = row_lse64(pm1, ps1, MT, lane < (int)C, a.tau64);
-      if (hasD) lse64D = row_lse64(pm2, ps2, MD, lane < (int)C, a.tau64);
-      if (x_ok) {
-        const uint32_t oa = peer_addr(&tl->xs[par], (uint32_t)(x / a.slice));
-        zxT = (double)ld_peer_f32(oa + 16);
-        zxD = (double)ld_peer_f32(oa + 20);
-      }
-    }
-
-    // Leader bookkeeping: TV of the previous row, lse / lp / log-weight of this one.
-    if (leader && warp == 0) {
-      if (prev_tv_idx >= 0) {
-        float acc = 0.f;
-        if (lane < nwarps)
-          for (int c = 0; c < (int)C; ++c) acc += tl->tvp[par ^ 1][c][lane];
-        acc = warp_sum(acc);
-        if (lane == 0) a.tv_out[prev_tv_idx] = prev_bad ? NAN : 0.5f * acc;
-      }
+    if (leader && warp == 0) {  // hand the row to the bookkeeping warp
+      const int slot = (int)(it % kLogN);
+      if (it >= kLogN && !mbar_wait(&tl->logempty[slot], (uint32_t)(((it / kLogN) - 1) & 1)))
+        raise_err(a.dev_err, SD_DEV_TIMEOUT);
+      if (lane < (int)C) tl->log[slot].m[lane] = rv[lane];
       if (lane == 0) {
-        if (bad && (!VERIFY || k < a.K || !done)) raise_err(a.dev_err, SD_DEV_NONFINITE);
-        if (!VERIFY) {
-          if (a.lse_out) {
-            a.lse_out[rowT * 2 + 0] = badT ? NAN : lse64T;
-            a.lse_out[rowT * 2 + 1] = badD ? NAN : lse64D;
-          }
-          if (k < a.K) {
-            double lp = NAN, lq = NAN;
-            if (!x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
-            if (x_ok && !bad) {
-              lp = zxT / a.tau64 - lse64T;
-              lq = zxD / a.tau64 - lse64D;
-            } else {
-              unit_bad = true;
-            }
-            logw_acc += lp - lq;
-            if (a.lp_out) {
-              a.lp_out[(unit * a.K + k) * 2 + 0] = lp;
-              a.lp_out[(unit * a.K + k) * 2 + 1] = lq;
-            }
-          }
-        }
+        tl->log[slot].unit = unit;
+        tl->log[slot].k = k;
+        tl->log[slot].x = x;
       }
-    }
-    const bool want_tv = hasD && a.tv_out != nullptr;
-    if (leader && warp == 0) {
-      prev_tv_idx = want_tv ? (VERIFY ? rowD : rowT) : -1;
-      prev_bad = bad;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->logfull[slot]);
     }
 
     // Per-warp scales turning register exps into normalised probabilities.
     const float scT = (mwT > -INFINITY && !badT) ? ex2((mwT - MT) * a.cT) / ST : 0.f;
     const float scD = (hasD && mwD > -INFINITY && !badD) ? ex2((mwD - MD) * a.cT) / SD : 0.f;
 
-    if (want_tv) {
+    if (want_tv && hasD) {
       float tv = 0.f;
 #pragma unroll
       for (int i = 0; i < EPT; ++i) tv += fabsf(__fmul_rn(xt[i], scT) - __fmul_rn(xd[i], scD));
       tv = warp_sum(tv);
-      if (lane == 0) st_peer_f32(peer_addr(&tl->tvp[par][rank][warp], 0), tv);
+      if (lane == 0) tl->tvw[warp] = tv;
     }
 
-    // ---------------- verification: accept test (CTA-uniform, fp64) ----------------
+    // ---------------- verification: accept test (identical in every CTA, fp64) ----------------
     bool draw_residual = false;
     if (VERIFY && k < a.K && !done) {
-      if (warp == 0 && lane == 0) {
-        int acc = 0;
-        if (!bad && x_ok)
-          acc = accept_test(zxT, zxD, lse64T, lse64D, a.tau64, a.seed, a.round, (uint32_t)rowT);
-        tl->flag[0] = acc;
-        tl->lse64[0] = lse64T;
-        tl->lse64[1] = lse64D;
-        if (leader && !x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
+      if (warp == 0) {
+        const double lse64T = row_lse64(pm1, ps1, MT, lane < (int)C, a.tau64);
+        const double lse64D = row_lse64(pm2, ps2, MD, lane < (int)C, a.tau64);
+        if (lane == 0) {
+          int acc = 0;
+          if (!bad && x_ok) {
+            const Msg& o = rv[x / a.slice];
+            acc = accept_test((double)o.zxT, (double)o.zxD, lse64T, lse64D, a.tau64, a.seed,
+                              a.round, (uint32_t)rowT);
+          }
+          tl->flag[0] = acc;
+          tl->lse64[0] = lse64T;
+          tl->lse64[1] = lse64D;
+          if (leader && !x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
+          if (leader && bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
+        }
       }
-      __syncthreads();
+      bar_sync_n(ncomp);
       const bool accept = tl->flag[0] != 0;
       if (bad) {
         done = true;
@@ -685,23 +821,31 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
       } else {
         draw_residual = true;
       }
+    } else if (VERIFY && bad && leader && tid == 0 && (k < a.K || !done)) {
+      raise_err(a.dev_err, SD_DEV_NONFINITE);
     }
 
     // ---------------- Gumbel-max draws: bonus token / residual token ----------------
     const bool draw_bonus = (k == a.K) && !badT && (!VERIFY || !done);
     if (draw_bonus || draw_residual) {
+      // Reference entry: the row's argmax v* (first CTA with the row max).
+      int vstar = 0x7FFFFFFF;
+      {
+        const bool mine = lane < (int)C && pm1 == MT;
+        int cand = mine ? rv[lane].aux : 0x7FFFFFFF;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
+        vstar = cand;
+      }
       ScreenCtx cx;
       cx.s0 = s0;
       cx.len = len;
       cx.tid = tid;
-      cx.nthr = nthr;
+      cx.nthr = ncomp;
       cx.gT = gT;
       cx.gD = gD;
       cx.tau64 = a.tau64;
       cx.mw_a = mwTs * a.inv_tau;
-      // Tref = M/tau + g_min - margin <= exact score of the row's max entry.
-      const float margin = 1e-5f + 2e-7f * fabsf(MT * a.inv_tau);
-      cx.rho = (mwT > -INFINITY) ? ex2((mwT - MT) * a.cT + (-kGumbelMinF + margin) * kLog2e) : 0.f;
       cx.scT = scT;
       cx.scD = scD;
       cx.mwT = mwTs;
@@ -714,10 +858,18 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
       const uint32_t tag = draw_bonus ? SD_STREAM_BONUS : SD_STREAM_RESIDUAL;
       cx.rowid = draw_bonus ? (uint32_t)unit : (uint32_t)rowT;
       const Stream st(a.seed, a.round, tag);
+      // Tref = fp32 score of v* minus its error bound: a lower bound on the winner.
+      {
+        const U4 w = st.at((uint32_t)(vstar >> 2), cx.rowid);
+        const float g = gumbel_f32(uniform_f32(word_of(w, vstar & 3)));
+        const float av = MT * a.inv_tau;
+        const float margin = 4e-6f + 1e-6f * (fabsf(av) + 2.f * fabsf(g));
+        cx.rho = (mwT > -INFINITY) ? ex2((mwT - MT) * a.cT + (margin - g) * kLog2e) : 0.f;
+      }
       int mode = draw_bonus ? 0 : 1;
       for (int pass = 0; pass < 2; ++pass) {
-        // pass 0: residual (mode 1) or bonus (mode 0); pass 1 only for an
-        // all-zero residual: draw from p with the same stream.
+        const int up = uses & 1;
+        ++uses;
         Cand cd = cand_empty();
         if (!VERIFY)
           screen<CPT, EPC, 0>(xt, xd, cx, st, cd);
@@ -725,73 +877,60 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
           screen_global<TIn, CPT>(cx, st, mode, &cd);
         cd = warp_cand(cd);
         if (lane == 0) tl->wcand[warp] = cd;
-        __syncthreads();
+        bar_sync_n(ncomp);
         if (warp == 0) {
           Cand c2 = lane < nwarps ? tl->wcand[lane] : cand_empty();
           c2 = warp_cand(c2);
-          if (lane == 0) tl->xc = c2;
-        }
-        cluster_sync();  // (C1)
-        if (warp == 0) {
-          Cand c3 = cand_empty();
+          if (lane == 0) mbar_arrive_expect_tx(&tl->cbar[up], C * (uint32_t)sizeof(Cand));
           if (lane < (int)C) {
-            const uint32_t pa = peer_addr(&tl->xc, lane);
-            c3.s = ld_peer_f32(pa + 0);
-            c3.lo = ld_peer_f32(pa + 4);
-            c3.hi = ld_peer_f32(pa + 8);
-            c3.ohi = ld_peer_f32(pa + 12);
-            c3.idx = ld_peer_s32(pa + 16);
-          }
-          c3 = warp_cand(c3);
-          if (lane == 0) {
-            const bool none = c3.idx == 0x7FFFFFFF;
-            tl->flag[1] = none ? 2 : (c3.ohi < c3.lo ? 0 : 1);  // 0 clear, 1 near-tie, 2 nothing
-            tl->flag[2] = c3.idx;
-            reinterpret_cast<float*>(&tl->flag[3])[0] = c3.lo;
+            const uint32_t ra = peer_addr(&tl->crecv[up][rank], (uint32_t)lane);
+            const uint32_t rb = peer_addr(&tl->cbar[up], (uint32_t)lane);
+            st_async_v4(ra, c2.s, c2.lo, c2.hi, c2.ohi, rb);
+            st_async_v4(ra + 16, __int_as_float(c2.idx), 0.f, 0.f, 0.f, rb);
           }
         }
-        __syncthreads();
-        const int decision = tl->flag[1];
-        int winner = tl->flag[2];
-        if (decision == 2 && mode == 1) {  // all-zero residual: sample p instead
+        if (!mbar_wait(&tl->cbar[up], (uint32_t)(((uses - 1) >> 1) & 1)))
+          raise_err(a.dev_err, SD_DEV_TIMEOUT);
+        Cand c3 = lane < (int)C ? tl->crecv[up][lane] : cand_empty();
+        c3 = warp_cand(c3);
+        const int decision = c3.idx == 0x7FFFFFFF ? 2 : (c3.ohi < c3.lo ? 0 : 1);
+        int winner = c3.idx;
+        if (decision == 2 && mode == 1) {  // all-zero residual: draw from p instead
           if (leader && tid == 0) raise_err(a.dev_err, SD_DEV_ZERO_RESIDUAL);
           mode = 0;
           continue;
         }
         if (decision == 1) {  // near-tie: exact fp64 re-score of every entry that can still win
-          const float lo_star = reinterpret_cast<const float*>(&tl->flag[3])[0];
+          const int dp = duses & 1;
+          const uint32_t dph = (uint32_t)((duses >> 1) & 1);
+          ++duses;
           double s64 = -INFINITY;
           int i64 = 0x7FFFFFFF;
-          rescore_exact<TIn, CPT>(cx, st, mode, lo_star, &s64, &i64);
+          rescore_exact<TIn, CPT>(cx, st, mode, c3.lo, &s64, &i64);
           warp_c64(s64, i64);
           if (lane == 0) {
             tl->wc64[warp].s = s64;
             tl->wc64[warp].idx = i64;
           }
-          __syncthreads();
+          bar_sync_n(ncomp);
           if (warp == 0) {
             double ss = lane < nwarps ? tl->wc64[lane].s : -INFINITY;
             int ii = lane < nwarps ? tl->wc64[lane].idx : 0x7FFFFFFF;
             warp_c64(ss, ii);
-            if (lane == 0) {
-              tl->xc64.s = ss;
-              tl->xc64.idx = ii;
-            }
-          }
-          cluster_sync();  // (C2)
-          if (warp == 0) {
-            double ss = -INFINITY;
-            int ii = 0x7FFFFFFF;
+            if (lane == 0) mbar_arrive_expect_tx(&tl->dbar[dp], C * (uint32_t)sizeof(Cand64));
             if (lane < (int)C) {
-              const uint32_t pa = peer_addr(&tl->xc64, lane);
-              ss = ld_peer_f64(pa);
-              ii = ld_peer_s32(pa + 8);
+              const uint32_t ra = peer_addr(&tl->drecv[dp][rank], (uint32_t)lane);
+              const uint32_t rb = peer_addr(&tl->dbar[dp], (uint32_t)lane);
+              const unsigned long long bits = __double_as_longlong(ss);
+              st_async_v4(ra, __uint_as_float((uint32_t)bits), __uint_as_float((uint32_t)(bits >> 32)),
+                          __int_as_float(ii), 0.f, rb);
             }
-            warp_c64(ss, ii);
-            if (lane == 0) tl->flag[2] = ii;
           }
-          __syncthreads();
-          winner = tl->flag[2];
+          if (!mbar_wait(&tl->dbar[dp], dph)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+          double ss = lane < (int)C ? tl->drecv[dp][lane].s : -INFINITY;
+          int ii = lane < (int)C ? tl->drecv[dp][lane].idx : 0x7FFFFFFF;
+          warp_c64(ss, ii);
+          winner = ii;
           if (winner == 0x7FFFFFFF && mode == 1) {  // exact residual is zero everywhere
             if (leader && tid == 0) raise_err(a.dev_err, SD_DEV_ZERO_RESIDUAL);
             mode = 0;
@@ -811,17 +950,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
       }
     }
 
-    // ---------------- end of unit: write per-particle / per-sequence outputs ----------------
+    // ---------------- end of unit ----------------
     if (k == a.K && leader && tid == 0) {
       if (!VERIFY) {
         if (badT) {
           a.bonus_out[unit] = -1;
           if (a.tokens_out) a.tokens_out[unit * a.R + a.K] = -1;
         }
-        const double prev = a.logw_prev ? a.logw_prev[unit] : 0.0;
-        a.logw_out[unit] = unit_bad ? NAN : prev + logw_acc;
-        if (a.tokens_out)
-          for (int j = 0; j < a.K; ++j) a.tokens_out[unit * a.R + j] = a.draft[unit * a.K + j];
       } else {
         a.acc_len[unit] = acc_len;
         for (int j = 0; j < a.R; ++j) {
@@ -834,15 +969,27 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     }
   }
 
-  cluster_sync();  // (F) last row's TV partials are in; no peer reads our smem after this
-  if (leader && warp == 0 && prev_tv_idx >= 0) {
-    const int par = (int)((nrows - 1) & 1);
-    float acc = 0.f;
-    if (lane < nwarps)
-      for (int c = 0; c < (int)C; ++c) acc += tl->tvp[par][c][lane];
-    acc = warp_sum(acc);
-    if (lane == 0) a.tv_out[prev_tv_idx] = prev_bad ? NAN : 0.5f * acc;
+  // Last row's TV partials go to the leader, which hands them to its bookkeeping warp.
+  if (want_tv && nrows > 0) {
+    bar_sync_n(ncomp);
+    if (warp == 0) {
+      float tvp = lane < nwarps ? tl->tvw[lane] : 0.f;
+      tvp = warp_sum(tvp);
+      if (leader && lane == 0) mbar_arrive_expect_tx(&tl->fbar, C * 4u);
+      if (lane == 0)
+        st_async_b32(peer_addr(&tl->frecv[rank], 0), __float_as_uint(tvp), peer_addr(&tl->fbar, 0));
+      if (leader) {
+        if (!mbar_wait(&tl->fbar, 0)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+        const int slot = (int)(nrows % kLogN);
+        if (nrows >= kLogN && !mbar_wait(&tl->logempty[slot], (uint32_t)(((nrows / kLogN) - 1) & 1)))
+          raise_err(a.dev_err, SD_DEV_TIMEOUT);
+        if (lane < (int)C) tl->log[slot].m[lane].tvprev = tl->frecv[lane];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tl->logfull[slot]);
+      }
+    }
   }
+  cluster_sync();  // all messages into this CTA have landed; peers may exit
 }
 
 // ------------------------------------------------------------------ host side
@@ -904,7 +1051,8 @@ static bool make_plan(const void* fn, int V, int esize, int64_t units, LaunchPla
   int64_t best_score = -1;
   for (int C = 1; C <= kMaxCluster; ++C) {
     const int slice = (int)(((int64_t)(V + C - 1) / C + 7) / 8 * 8);
-    const int threads = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
+    const int compute = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
+    const int threads = compute + 32;  // + the bookkeeping warp
     if (threads > kMaxThreads) continue;
     const uint32_t sb = (uint32_t)(((int64_t)slice * esize + 127) / 128 * 128);
     int stages = 0;

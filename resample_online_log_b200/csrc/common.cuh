@@ -225,9 +225,9 @@ __device__ __forceinline__ void st_async_b32(uint32_t raddr, uint32_t v, uint32_
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
-// Barrier among the first `n` threads of the CTA (id 1; id 0 is __syncthreads).
-__device__ __forceinline__ void bar_sync_n(int n) {
-  asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory");
+// Named barrier `id` (1..15; 0 is __syncthreads) among `n` threads.
+__device__ __forceinline__ void bar_sync_n(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 __device__ __forceinline__ void raise_err(uint32_t* dev_err, uint32_t bits) {

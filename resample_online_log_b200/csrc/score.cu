@@ -30,6 +30,7 @@
 //     the entries that can still win (most are pruned before any Philox call
 //     or log), and near-ties are re-scored in fp64 from the logits in HBM.
 #include <cstdio>
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -50,7 +51,8 @@ struct ScoreArgs {
   int64_t ld;
   int V, K, R;
   int64_t units;
-  int slice;
+  int slice;             // entries per group slice (a multiple of 8)
+  int groups;            // independent warp groups per CTA (1..3)
   int stages;
   uint32_t stage_bytes;  // bytes reserved for one tensor's slice in a stage
   int use_tma;
@@ -80,32 +82,26 @@ struct Cand64 {
   int idx, pad;
 };
 
-// One CTA's message for one row, pushed into every CTA of the cluster.
+constexpr int kMaxGroups = 3;
+constexpr int kMaxSlices = 32;  // cluster size x groups
+
+// One group's message for one row, pushed into every CTA of the cluster.
 struct alignas(16) Msg {
   float mT, sT, mD, sD;  // (max, sum of exps relative to it) over its slice of each row
-  float zxT, zxD;        // raw logits of the draft token (owner CTA only)
-  float tvprev;          // this CTA's TV partial of its previous row
+  float zxT, zxD;        // raw logits of the draft token (owner slice only)
+  float tvprev;          // this group's TV partial of its previous row
   int aux;               // argmax entry of its target slice (rows that draw a token)
 };
 
 constexpr int kLogN = 4;
-// Row record handed from the leader's compute warps to its bookkeeping warp.
+// Row record handed from the leader's group 0 to its bookkeeping warp.
 struct alignas(16) LogEntry {
-  Msg m[kMaxCluster];
+  Msg m[kMaxSlices];
   int64_t unit;
   int k, x;
 };
 
-struct alignas(128) Tail {
-  uint64_t full[4];           // ring stages (bulk copies)
-  uint64_t rbar[2];           // row messages, by row parity
-  uint64_t cbar[2], dbar[2];  // candidate / fp64 messages, by use parity
-  uint64_t fbar, pad_bar;
-  uint64_t logfull[kLogN], logempty[kLogN];
-  Msg recv[2][kMaxCluster];
-  Cand crecv[2][kMaxCluster];
-  Cand64 drecv[2][kMaxCluster];
-  float frecv[kMaxCluster];
+struct alignas(16) GroupState {  // scratch of one warp group
   float4 wpart[kMaxWarps];
   float tvw[kMaxWarps];
   float wargv[kMaxWarps];
@@ -115,6 +111,21 @@ struct alignas(128) Tail {
   float zx[2][2];
   double lse64[2];
   int flag[4];
+};
+
+struct alignas(128) Tail {
+  uint64_t full[4];           // ring stages (bulk copies)
+  uint64_t rbar[2];           // row messages, by row parity
+  uint64_t cbar[2], dbar[2];  // candidate / fp64 messages, by use parity
+  uint64_t fbar, pad_bar;
+  uint64_t logfull[kLogN], logempty[kLogN];
+  int stage_cnt[4];           // groups done with each stage
+  int pad_cnt[4];
+  Msg recv[2][kMaxSlices];
+  Cand crecv[2][kMaxSlices];
+  Cand64 drecv[2][kMaxSlices];
+  float frecv[kMaxSlices];
+  GroupState gs[kMaxGroups];
   LogEntry log[kLogN];
 };
 
@@ -276,64 +287,6 @@ __device__ __forceinline__ bool keep_bonus(float y, float u) {
   return y > 0.f && !(u < (1.0f - y * 1.001f) - 2.4e-7f);
 }
 
-template <int CPT, int EPC, int MODE>
-__device__ __forceinline__ void screen(const float* xt, const float* xd, const ScreenCtx& cx,
-                                       const Stream& st, Cand& out) {
-#pragma unroll
-  for (int c = 0; c < CPT; ++c) {
-    const int e0 = (cx.tid + c * cx.nthr) * EPC;
-    if (e0 >= cx.len) continue;
-#pragma unroll
-    for (int gq = 0; gq < EPC / 4; ++gq) {
-      const int base = c * EPC + gq * 4;
-      const int v0 = cx.s0 + e0 + gq * 4;
-      float y[4], r[4], eb[4];
-      float ymax = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (MODE == 0) {
-          y[j] = xt[base + j] * cx.rho;
-          ymax = fmaxf(ymax, y[j]);
-        } else {
-          const float p = xt[base + j] * cx.scT, q = xd[base + j] * cx.scD;
-          r[j] = p - q;
-          eb[j] = 7.7e-6f * (p + q);  // > 2^-17 (p + q): fp32 error bound of p - q
-          ymax = fmaxf(ymax, r[j] + eb[j]);
-        }
-      }
-      if (MODE == 0 ? (ymax < kYSkip) : !(ymax > 0.f)) continue;
-      const U4 w = st.at((uint32_t)(v0 >> 2), cx.rowid);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (e0 + gq * 4 + j >= cx.len) continue;
-        const float u = uniform_f32(word_of(w, j));
-        Cand cd;
-        if (MODE == 0) {
-          if (!keep_bonus(y[j], u)) continue;
-          const float g32 = gumbel_f32(u);
-          const float a32 = cx.mw_a + logf(xt[base + j]);
-          cd.s = a32 + g32;
-          const float d = 4e-6f + 4.8e-7f * (fabsf(a32) + 2.f * fabsf(g32));
-          cd.lo = cd.s - d;
-          cd.hi = cd.s + d;
-        } else {
-          if (!(r[j] + eb[j] > 0.f)) continue;
-          const float g32 = gumbel_f32(u);
-          const float lh = logf(r[j] + eb[j]);
-          const float d = 4e-6f + 4.8e-7f * (fabsf(lh) + 2.f * fabsf(g32));
-          cd.hi = lh + g32 + d;
-          cd.s = r[j] > 0.f ? logf(r[j]) + g32 : -INFINITY;
-          cd.lo = r[j] - eb[j] > 0.f ? logf(r[j] - eb[j]) + g32 - d : -INFINITY;
-        }
-        cd.ohi = -INFINITY;
-        cd.idx = v0 + j;
-        cd.pad0 = cd.pad1 = cd.pad2 = 0;
-        out = cand_merge(out, cd);
-      }
-    }
-  }
-}
-
 // Exact fp64 maximum over the entries the screen keeps whose upper bound
 // reaches lo_star.  Recomputes the screen's fp32 values from the logits in HBM
 // (same operations, same inputs, so the same entries are kept) and scores the
@@ -479,22 +432,77 @@ __device__ __noinline__ int accept_test(double zxT, double zxD, double lseT, dou
 }
 
 // ------------------------------------------------------------------ the kernel
-// Message exchange: after its CTA-level reduction a CTA pushes one 32-byte Msg
-// into slot [rank] of every CTA of the cluster with st.async, which completes
-// transaction bytes on the receiver's mbarrier; each CTA arms its own barrier
-// for C messages and waits on it.  No cluster-wide barrier and no fence sits
-// on the per-row path.  Slots and barriers alternate by row parity: a CTA can
-// only send row r+2 after it has every row r+1 message, and every CTA reads
-// its row r slots before sending row r+1, so a slot is never overwritten
-// before it is read.
+// Work split: a cluster of C CTAs scores one row pair at a time; each CTA runs
+// `groups` independent warp groups, and group g of CTA q owns vocabulary slice
+// j = q*groups + g (J = C*groups slices per row).  The groups of a CTA share the
+// bulk-copy ring but otherwise run unsynchronised, so one group's exp2 phase
+// overlaps another group's exchange, TV and bookkeeping of the same or the
+// previous row (ping-pong), which keeps MUFU and the issue slots busy.
+//
+// Message exchange: after its group-level reduction a group pushes one 32-byte
+// Msg into slot [j] of every CTA of the cluster with st.async, which completes
+// transaction bytes on the receiver's mbarrier; group 0 of each CTA arms the
+// CTA's barrier for J messages per row and every group waits on it.  No
+// cluster-wide barrier or fence sits on the per-row path.  Slots and barriers
+// alternate by row parity: a group can only send row r+2 after every group has
+// sent row r+1, which each does only after reading its row r slots.
 
-__device__ __forceinline__ void send_row_msg(Tail* tl, int par, uint32_t rank, uint32_t C, int lane,
+__device__ __forceinline__ void send_row_msg(Tail* tl, int par, int j, uint32_t C, int lane,
                                              const Msg& m) {
-  if (lane < (int)C) {
-    const uint32_t ra = peer_addr(&tl->recv[par][rank], (uint32_t)lane);
+  if (lane < (int)C) {  // lane l -> slot j of CTA l
+    const uint32_t ra = peer_addr(&tl->recv[par][j], (uint32_t)lane);
     const uint32_t rb = peer_addr(&tl->rbar[par], (uint32_t)lane);
     st_async_v4(ra, m.mT, m.sT, m.mD, m.sD, rb);
     st_async_v4(ra + 16, m.zxT, m.zxD, m.tvprev, __int_as_float(m.aux), rb);
+  }
+}
+
+// Candidate scoring of one kept entry (rare; kept out of line to keep the hot
+// loop small).
+__device__ __noinline__ Cand bonus_cand(float e, float u, float mw_a, int v) {
+  const float g32 = gumbel_f32(u);
+  const float a32 = mw_a + logf(e);
+  Cand cd;
+  cd.s = a32 + g32;
+  const float d = 4e-6f + 4.8e-7f * (fabsf(a32) + 2.f * fabsf(g32));
+  cd.lo = cd.s - d;
+  cd.hi = cd.s + d;
+  cd.ohi = -INFINITY;
+  cd.idx = v;
+  cd.pad0 = cd.pad1 = cd.pad2 = 0;
+  return cd;
+}
+
+// Register screen for the bonus token (SMC-SD): entries of this thread, exps
+// xt relative to its warp max; see the Gumbel-screen notes above.
+template <int CPT, int EPC>
+__device__ __forceinline__ void screen_bonus(const float* xt, const ScreenCtx& cx,
+                                             const Stream& st, Cand& out) {
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) {
+    const int e0 = (cx.tid + c * cx.nthr) * EPC;
+    if (e0 >= cx.len) continue;
+#pragma unroll
+    for (int gq = 0; gq < EPC / 4; ++gq) {
+      const int base = c * EPC + gq * 4;
+      const int v0 = cx.s0 + e0 + gq * 4;
+      const float y0 = xt[base] * cx.rho, y1 = xt[base + 1] * cx.rho;
+      const float y2 = xt[base + 2] * cx.rho, y3 = xt[base + 3] * cx.rho;
+      if (fmaxf(fmaxf(y0, y1), fmaxf(y2, y3)) < kYSkip) continue;
+      const U4 w = st.at((uint32_t)(v0 >> 2), cx.rowid);
+      const float u0 = uniform_f32(w.x), u1 = uniform_f32(w.y);
+      const float u2 = uniform_f32(w.z), u3 = uniform_f32(w.w);
+      const bool k0 = keep_bonus(y0, u0) && e0 + gq * 4 + 0 < cx.len;
+      const bool k1 = keep_bonus(y1, u1) && e0 + gq * 4 + 1 < cx.len;
+      const bool k2 = keep_bonus(y2, u2) && e0 + gq * 4 + 2 < cx.len;
+      const bool k3 = keep_bonus(y3, u3) && e0 + gq * 4 + 3 < cx.len;
+      if (k0 | k1 | k2 | k3) {
+        if (k0) out = cand_merge(out, bonus_cand(xt[base], u0, cx.mw_a, v0));
+        if (k1) out = cand_merge(out, bonus_cand(xt[base + 1], u1, cx.mw_a, v0 + 1));
+        if (k2) out = cand_merge(out, bonus_cand(xt[base + 2], u2, cx.mw_a, v0 + 2));
+        if (k3) out = cand_merge(out, bonus_cand(xt[base + 3], u3, cx.mw_a, v0 + 3));
+      }
+    }
   }
 }
 
@@ -502,8 +510,7 @@ __device__ __forceinline__ void send_row_msg(Tail* tl, int par, uint32_t rank, u
 // per-particle outputs, fed row by row through a small shared-memory ring so
 // that none of this sits on the compute warps' critical path.
 template <bool VERIFY>
-__device__ void bookkeep(const ScoreArgs& a, Tail* tl, uint32_t C, uint32_t cid, uint32_t G,
-                         int64_t nrows, bool want_tv) {
+__device__ void bookkeep(const ScoreArgs& a, Tail* tl, uint32_t J, int64_t nrows, bool want_tv) {
   const int lane = threadIdx.x & 31;
   double logw_acc = 0.0;
   bool unit_bad = false;
@@ -515,8 +522,8 @@ __device__ void bookkeep(const ScoreArgs& a, Tail* tl, uint32_t C, uint32_t cid,
     if (!mbar_wait(&tl->logfull[slot], (uint32_t)((it / kLogN) & 1)))
       raise_err(a.dev_err, SD_DEV_TIMEOUT);
     const LogEntry& e = tl->log[slot];
-    if (prev_tv_idx >= 0) {  // every message carries its CTA's TV partial of the previous row
-      float v = lane < (int)C ? e.m[lane].tvprev : 0.f;
+    if (prev_tv_idx >= 0) {  // every message carries its group's TV partial of the previous row
+      float v = lane < (int)J ? e.m[lane].tvprev : 0.f;
       v = warp_sum(v);
       if (lane == 0) a.tv_out[prev_tv_idx] = prev_bad ? NAN : 0.5f * v;
     }
@@ -528,10 +535,10 @@ __device__ void bookkeep(const ScoreArgs& a, Tail* tl, uint32_t C, uint32_t cid,
     const int64_t unit = e.unit;
     const int k = e.k, x = e.x;
     const bool hasD = !VERIFY || k < a.K;
-    const float pm1 = lane < (int)C ? e.m[lane].mT : -INFINITY;
-    const float ps1 = lane < (int)C ? e.m[lane].sT : 0.f;
-    const float pm2 = lane < (int)C ? e.m[lane].mD : -INFINITY;
-    const float ps2 = lane < (int)C ? e.m[lane].sD : 0.f;
+    const float pm1 = lane < (int)J ? e.m[lane].mT : -INFINITY;
+    const float ps1 = lane < (int)J ? e.m[lane].sT : 0.f;
+    const float pm2 = lane < (int)J ? e.m[lane].mD : -INFINITY;
+    const float ps2 = lane < (int)J ? e.m[lane].sD : 0.f;
     const float MT = warp_max(pm1);
     const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
     const float MD = hasD ? warp_max(pm2) : 0.f;
@@ -546,8 +553,8 @@ __device__ void bookkeep(const ScoreArgs& a, Tail* tl, uint32_t C, uint32_t cid,
         logw_acc = 0.0;
         unit_bad = false;
       }
-      const double lse64T = row_lse64(pm1, ps1, MT, lane < (int)C, a.tau64);
-      const double lse64D = row_lse64(pm2, ps2, MD, lane < (int)C, a.tau64);
+      const double lse64T = row_lse64(pm1, ps1, MT, lane < (int)J, a.tau64);
+      const double lse64D = row_lse64(pm2, ps2, MD, lane < (int)J, a.tau64);
       if (lane == 0) {
         if (bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
         if (a.lse_out) {
@@ -574,7 +581,8 @@ __device__ void bookkeep(const ScoreArgs& a, Tail* tl, uint32_t C, uint32_t cid,
           const double prev = a.logw_prev ? a.logw_prev[unit] : 0.0;
           a.logw_out[unit] = unit_bad ? NAN : prev + logw_acc;
           if (a.tokens_out)
-            for (int j = 0; j < a.K; ++j) a.tokens_out[unit * a.R + j] = a.draft[unit * a.K + j];
+            for (int jj = 0; jj < a.K; ++jj)
+              a.tokens_out[unit * a.R + jj] = a.draft[unit * a.K + jj];
         }
       }
     }
@@ -593,22 +601,35 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ncomp = blockDim.x - 32, nwarps = ncomp >> 5;  // last warp: bookkeeping
+  const int ncomp = blockDim.x - 32;          // last warp: service (bookkeeping)
+  const uint32_t NG = (uint32_t)a.groups;
+  const int gthr = ncomp / (int)NG;           // threads per group
+  const int grp = tid / gthr;                 // this thread's group (== NG for the service warp)
+  const int gtid = tid - grp * gthr, gwarp = gtid >> 5, gnw = gthr >> 5;
   const uint32_t rank = cluster_rank(), C = cluster_size();
   const uint32_t cid = cluster_id(), G = num_clusters();
+  const uint32_t J = C * NG;
   Tail* tl = reinterpret_cast<Tail*>(smem + (size_t)a.stages * 2 * a.stage_bytes);
 
-  const int s0 = (int)rank * a.slice;
+  // This CTA's vocabulary range (copied by bulk copies) and this group's slice.
+  const int cs0 = (int)rank * (int)NG * a.slice;
+  const int clen = max(0, min((int)NG * a.slice, a.V - cs0));
+  const int ctma = a.use_tma ? ((clen * (int)sizeof(TIn)) & ~15) / (int)sizeof(TIn) : 0;
+  const uint32_t tma_bytes = (uint32_t)ctma * (uint32_t)sizeof(TIn);
+  const int jslice = (int)rank * (int)NG + grp;
+  const int s0 = jslice * a.slice;
   const int len = max(0, min(a.slice, a.V - s0));
-  const int tma_len = a.use_tma ? ((len * (int)sizeof(TIn)) & ~15) / (int)sizeof(TIn) : 0;
-  const uint32_t tma_bytes = (uint32_t)tma_len * (uint32_t)sizeof(TIn);
+  const int tma_len = max(0, min(len, ctma - grp * a.slice));  // entries of the slice in smem
   const int64_t my_units = (int64_t)cid < a.units ? (a.units - 1 - cid) / G + 1 : 0;
   const int64_t nrows = my_units * a.R;
   const bool leader = rank == 0;
   const bool want_tv = a.tv_out != nullptr;
 
   if (tid == 0) {
-    for (int s = 0; s < a.stages; ++s) mbar_init(&tl->full[s], 1);
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&tl->full[s], 1);
+      tl->stage_cnt[s] = 0;
+    }
     for (int p = 0; p < 2; ++p) {
       mbar_init(&tl->rbar[p], 1);
       mbar_init(&tl->cbar[p], 1);
@@ -624,12 +645,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
   __syncthreads();
   cluster_sync();  // every CTA's barriers exist before anyone sends to them
 
-  if (warp == nwarps) {
-    if (leader) bookkeep<VERIFY>(a, tl, C, cid, G, nrows, want_tv);
+  if (warp == ncomp / 32) {
+    if (leader) bookkeep<VERIFY>(a, tl, J, nrows, want_tv);
     cluster_sync();
     return;
   }
 
+  GroupState* gs = &tl->gs[grp];
+  const int barid = 1 + grp;
   const uint64_t pol = policy_evict_first();
   auto issue = [&](int64_t it) {
     const int s = (int)(it % a.stages);
@@ -641,20 +664,20 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     unsigned char* stg = smem + (size_t)s * 2 * a.stage_bytes;
     mbar_arrive_expect_tx(&tl->full[s], tma_bytes * (hasD ? 2u : 1u));
     if (tma_bytes) {
-      bulk_load(stg, (const TIn*)a.zT + rowT * a.ld + s0, tma_bytes, &tl->full[s], pol);
+      bulk_load(stg, (const TIn*)a.zT + rowT * a.ld + cs0, tma_bytes, &tl->full[s], pol);
       if (hasD)
-        bulk_load(stg + a.stage_bytes, (const TIn*)a.zD + rowD * a.ld + s0, tma_bytes, &tl->full[s],
-                  pol);
+        bulk_load(stg + a.stage_bytes, (const TIn*)a.zD + rowD * a.ld + cs0, tma_bytes,
+                  &tl->full[s], pol);
     }
   };
   if (tid == 0)
     for (int64_t it = 0; it < nrows && it < a.stages; ++it) issue(it);
 
-  bool done = false;  // verify: sequence finished (identical in every CTA)
+  bool done = false;  // verify: sequence finished (identical in every group)
   int acc_len = 0;
   int emitted = -1;
-  int uses = 0;       // candidate exchanges so far
-  int duses = 0;      // fp64 exchanges so far
+  int uses = 0;   // candidate exchanges so far
+  int duses = 0;  // fp64 exchanges so far
   int x_pref = (nrows > 0 && a.K > 0) ? a.draft[(int64_t)cid * a.K] : -1;
 
   float xt[EPT], xd[EPT];
@@ -683,27 +706,38 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     }
 
     if (!mbar_wait(&tl->full[s], ph)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
-    const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)s * 2 * a.stage_bytes);
-    const TIn* stD =
-        reinterpret_cast<const TIn*>(smem + (size_t)s * 2 * a.stage_bytes + a.stage_bytes);
+    const TIn* stT =
+        reinterpret_cast<const TIn*>(smem + (size_t)s * 2 * a.stage_bytes) + grp * a.slice;
+    const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)s * 2 * a.stage_bytes +
+                                                  a.stage_bytes) + grp * a.slice;
     const TIn* gT = (const TIn*)a.zT + rowT * a.ld + s0;
     const TIn* gD = (const TIn*)a.zD + rowD * a.ld + s0;
 
-    const float mt = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, tid, ncomp);
+    const float mt = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, gtid, gthr);
     float md = -INFINITY;
-    if (hasD) md = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, tid, ncomp);
+    if (hasD) md = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, gtid, gthr);
+    const bool owner = x_ok && x >= s0 && x < s0 + len;
+    if (owner) {
+      const int le = x - s0;
+      if (((le / EPC) % gthr) == gtid) {
+        gs->zx[par][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
+        gs->zx[par][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
+      }
+    }
+    bar_sync_n(barid, gthr);  // (A0) this group is done with the stage
+    if (gtid == 0) {
+      // the last group to finish with the stage refills it
+      __threadfence_block();
+      if (atomicAdd(&tl->stage_cnt[s], 1) == (int)NG - 1) {
+        tl->stage_cnt[s] = 0;
+        if (it + a.stages < nrows) issue(it + a.stages);
+      }
+    }
     int amax = 0x7FFFFFFF;  // this thread's first entry equal to its max (global index)
     if (draws) {
 #pragma unroll
       for (int i = EPT - 1; i >= 0; --i)
-        if (xt[i] == mt) amax = s0 + (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
-    }
-    if (x_ok && x >= s0 && x < s0 + len) {
-      const int le = x - s0;
-      if (((le / EPC) % ncomp) == tid) {
-        tl->zx[par][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
-        tl->zx[par][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
-      }
+        if (xt[i] == mt) amax = s0 + (gtid + (i / EPC) * gthr) * EPC + (i % EPC);
     }
     const float mwT = warp_max(mt);
     const float mwD = hasD ? warp_max(md) : -INFINITY;
@@ -721,41 +755,41 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     sT = warp_sum(sT);
     if (hasD) sD = warp_sum(sD);
     if (lane == 0) {
-      tl->wpart[warp] = make_float4(mwT, sT, mwD, sD);
-      tl->wargv[warp] = mwT;
-      tl->wargi[warp] = amax;
+      gs->wpart[gwarp] = make_float4(mwT, sT, mwD, sD);
+      gs->wargv[gwarp] = mwT;
+      gs->wargi[gwarp] = amax;
     }
-    bar_sync_n(ncomp);  // (A) the stage is free; warp partials are visible
-    if (tid == 0 && it + a.stages < nrows) issue(it + a.stages);
-    if (warp == 0) {
+    bar_sync_n(barid, gthr);  // (A) warp partials are visible
+    if (gwarp == 0) {
       const float4 wp =
-          lane < nwarps ? tl->wpart[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+          lane < gnw ? gs->wpart[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
       Msg m;
       m.mT = warp_max(wp.x);
       m.mD = warp_max(wp.z);
       m.sT = warp_sum(part_term(wp.x, wp.y, m.mT, a.cT));
       m.sD = warp_sum(part_term(wp.z, wp.w, m.mD, a.cT));
-      float tvp = (lane < nwarps && it > 0) ? tl->tvw[lane] : 0.f;
+      const float tvp = (lane < gnw && it > 0) ? gs->tvw[lane] : 0.f;
       m.tvprev = warp_sum(tvp);
       int ai = 0x7FFFFFFF;
-      if (draws && lane < nwarps && tl->wargv[lane] == m.mT) ai = tl->wargi[lane];
+      if (draws) {
+        if (lane < gnw && gs->wargv[lane] == m.mT) ai = gs->wargi[lane];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ai = min(ai, __shfl_xor_sync(0xffffffffu, ai, o));
+        for (int o = 16; o > 0; o >>= 1) ai = min(ai, __shfl_xor_sync(0xffffffffu, ai, o));
+      }
       m.aux = ai;
-      const bool owner = x_ok && x >= s0 && x < s0 + len;
-      m.zxT = owner ? tl->zx[par][0] : 0.f;
-      m.zxD = owner ? tl->zx[par][1] : 0.f;
-      if (lane == 0) mbar_arrive_expect_tx(&tl->rbar[par], C * (uint32_t)sizeof(Msg));
-      send_row_msg(tl, par, rank, C, lane, m);
+      m.zxT = owner ? gs->zx[par][0] : 0.f;
+      m.zxD = owner ? gs->zx[par][1] : 0.f;
+      if (grp == 0 && lane == 0) mbar_arrive_expect_tx(&tl->rbar[par], J * (uint32_t)sizeof(Msg));
+      send_row_msg(tl, par, jslice, C, lane, m);
     }
     if (!mbar_wait(&tl->rbar[par], (uint32_t)((it >> 1) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
 
-    // Rebuild the row's normalisers from the C messages (every warp, same order).
+    // Rebuild the row's normalisers from the J messages (every warp, same order).
     const Msg* rv = tl->recv[par];
-    const float pm1 = lane < (int)C ? rv[lane].mT : -INFINITY;
-    const float ps1 = lane < (int)C ? rv[lane].sT : 0.f;
-    const float pm2 = lane < (int)C ? rv[lane].mD : -INFINITY;
-    const float ps2 = lane < (int)C ? rv[lane].sD : 0.f;
+    const float pm1 = lane < (int)J ? rv[lane].mT : -INFINITY;
+    const float ps1 = lane < (int)J ? rv[lane].sT : 0.f;
+    const float pm2 = lane < (int)J ? rv[lane].mD : -INFINITY;
+    const float ps2 = lane < (int)J ? rv[lane].sD : 0.f;
     const float MT = warp_max(pm1);
     const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
     const float MD = hasD ? warp_max(pm2) : 0.f;
@@ -764,11 +798,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     const bool badD = hasD && !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
     const bool bad = badT || badD;
 
-    if (leader && warp == 0) {  // hand the row to the bookkeeping warp
+    if (leader && grp == 0 && gwarp == 0) {  // hand the row to the bookkeeping warp
       const int slot = (int)(it % kLogN);
       if (it >= kLogN && !mbar_wait(&tl->logempty[slot], (uint32_t)(((it / kLogN) - 1) & 1)))
         raise_err(a.dev_err, SD_DEV_TIMEOUT);
-      if (lane < (int)C) tl->log[slot].m[lane] = rv[lane];
+      if (lane < (int)J) tl->log[slot].m[lane] = rv[lane];
       if (lane == 0) {
         tl->log[slot].unit = unit;
         tl->log[slot].k = k;
@@ -787,15 +821,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
 #pragma unroll
       for (int i = 0; i < EPT; ++i) tv += fabsf(__fmul_rn(xt[i], scT) - __fmul_rn(xd[i], scD));
       tv = warp_sum(tv);
-      if (lane == 0) tl->tvw[warp] = tv;
+      if (lane == 0) gs->tvw[gwarp] = tv;
     }
 
-    // ---------------- verification: accept test (identical in every CTA, fp64) ----------------
+    // ---------------- verification: accept test (identical in every group, fp64) ----------------
     bool draw_residual = false;
     if (VERIFY && k < a.K && !done) {
-      if (warp == 0) {
-        const double lse64T = row_lse64(pm1, ps1, MT, lane < (int)C, a.tau64);
-        const double lse64D = row_lse64(pm2, ps2, MD, lane < (int)C, a.tau64);
+      if (gwarp == 0) {
+        const double lse64T = row_lse64(pm1, ps1, MT, lane < (int)J, a.tau64);
+        const double lse64D = row_lse64(pm2, ps2, MD, lane < (int)J, a.tau64);
         if (lane == 0) {
           int acc = 0;
           if (!bad && x_ok) {
@@ -803,15 +837,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
             acc = accept_test((double)o.zxT, (double)o.zxD, lse64T, lse64D, a.tau64, a.seed,
                               a.round, (uint32_t)rowT);
           }
-          tl->flag[0] = acc;
-          tl->lse64[0] = lse64T;
-          tl->lse64[1] = lse64D;
-          if (leader && !x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
-          if (leader && bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
+          gs->flag[0] = acc;
+          gs->lse64[0] = lse64T;
+          gs->lse64[1] = lse64D;
+          if (leader && grp == 0 && !x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
+          if (leader && grp == 0 && bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
         }
       }
-      bar_sync_n(ncomp);
-      const bool accept = tl->flag[0] != 0;
+      bar_sync_n(barid, gthr);
+      const bool accept = gs->flag[0] != 0;
       if (bad) {
         done = true;
         acc_len = k;
@@ -828,11 +862,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
     // ---------------- Gumbel-max draws: bonus token / residual token ----------------
     const bool draw_bonus = (k == a.K) && !badT && (!VERIFY || !done);
     if (draw_bonus || draw_residual) {
-      // Reference entry: the row's argmax v* (first CTA with the row max).
-      int vstar = 0x7FFFFFFF;
+      // Reference entry: the row's argmax v* (first slice holding the row max).
+      int vstar;
       {
-        const bool mine = lane < (int)C && pm1 == MT;
-        int cand = mine ? rv[lane].aux : 0x7FFFFFFF;
+        int cand = (lane < (int)J && pm1 == MT) ? rv[lane].aux : 0x7FFFFFFF;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
         vstar = cand;
@@ -840,8 +873,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
       ScreenCtx cx;
       cx.s0 = s0;
       cx.len = len;
-      cx.tid = tid;
-      cx.nthr = ncomp;
+      cx.tid = gtid;
+      cx.nthr = gthr;
       cx.gT = gT;
       cx.gD = gD;
       cx.tau64 = a.tau64;
@@ -852,8 +885,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
       cx.mwD = mwDs;
       cx.cT = a.cT;
       if (draw_residual) {
-        cx.lseT = tl->lse64[0];
-        cx.lseD = tl->lse64[1];
+        cx.lseT = gs->lse64[0];
+        cx.lseD = gs->lse64[1];
       }
       const uint32_t tag = draw_bonus ? SD_STREAM_BONUS : SD_STREAM_RESIDUAL;
       cx.rowid = draw_bonus ? (uint32_t)unit : (uint32_t)rowT;
@@ -869,29 +902,29 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
       int mode = draw_bonus ? 0 : 1;
       for (int pass = 0; pass < 2; ++pass) {
         const int up = uses & 1;
+        const uint32_t uph = (uint32_t)((uses >> 1) & 1);
         ++uses;
         Cand cd = cand_empty();
         if (!VERIFY)
-          screen<CPT, EPC, 0>(xt, xd, cx, st, cd);
+          screen_bonus<CPT, EPC>(xt, cx, st, cd);
         else
           screen_global<TIn, CPT>(cx, st, mode, &cd);
         cd = warp_cand(cd);
-        if (lane == 0) tl->wcand[warp] = cd;
-        bar_sync_n(ncomp);
-        if (warp == 0) {
-          Cand c2 = lane < nwarps ? tl->wcand[lane] : cand_empty();
+        if (lane == 0) gs->wcand[gwarp] = cd;
+        bar_sync_n(barid, gthr);
+        if (gwarp == 0) {
+          Cand c2 = lane < gnw ? gs->wcand[lane] : cand_empty();
           c2 = warp_cand(c2);
-          if (lane == 0) mbar_arrive_expect_tx(&tl->cbar[up], C * (uint32_t)sizeof(Cand));
+          if (grp == 0 && lane == 0) mbar_arrive_expect_tx(&tl->cbar[up], J * (uint32_t)sizeof(Cand));
           if (lane < (int)C) {
-            const uint32_t ra = peer_addr(&tl->crecv[up][rank], (uint32_t)lane);
+            const uint32_t ra = peer_addr(&tl->crecv[up][jslice], (uint32_t)lane);
             const uint32_t rb = peer_addr(&tl->cbar[up], (uint32_t)lane);
             st_async_v4(ra, c2.s, c2.lo, c2.hi, c2.ohi, rb);
             st_async_v4(ra + 16, __int_as_float(c2.idx), 0.f, 0.f, 0.f, rb);
           }
         }
-        if (!mbar_wait(&tl->cbar[up], (uint32_t)(((uses - 1) >> 1) & 1)))
-          raise_err(a.dev_err, SD_DEV_TIMEOUT);
-        Cand c3 = lane < (int)C ? tl->crecv[up][lane] : cand_empty();
+        if (!mbar_wait(&tl->cbar[up], uph)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+        Cand c3 = lane < (int)J ? tl->crecv[up][lane] : cand_empty();
         c3 = warp_cand(c3);
         const int decision = c3.idx == 0x7FFFFFFF ? 2 : (c3.ohi < c3.lo ? 0 : 1);
         int winner = c3.idx;
@@ -909,26 +942,27 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
           rescore_exact<TIn, CPT>(cx, st, mode, c3.lo, &s64, &i64);
           warp_c64(s64, i64);
           if (lane == 0) {
-            tl->wc64[warp].s = s64;
-            tl->wc64[warp].idx = i64;
+            gs->wc64[gwarp].s = s64;
+            gs->wc64[gwarp].idx = i64;
           }
-          bar_sync_n(ncomp);
-          if (warp == 0) {
-            double ss = lane < nwarps ? tl->wc64[lane].s : -INFINITY;
-            int ii = lane < nwarps ? tl->wc64[lane].idx : 0x7FFFFFFF;
+          bar_sync_n(barid, gthr);
+          if (gwarp == 0) {
+            double ss = lane < gnw ? gs->wc64[lane].s : -INFINITY;
+            int ii = lane < gnw ? gs->wc64[lane].idx : 0x7FFFFFFF;
             warp_c64(ss, ii);
-            if (lane == 0) mbar_arrive_expect_tx(&tl->dbar[dp], C * (uint32_t)sizeof(Cand64));
+            if (grp == 0 && lane == 0)
+              mbar_arrive_expect_tx(&tl->dbar[dp], J * (uint32_t)sizeof(Cand64));
             if (lane < (int)C) {
-              const uint32_t ra = peer_addr(&tl->drecv[dp][rank], (uint32_t)lane);
+              const uint32_t ra = peer_addr(&tl->drecv[dp][jslice], (uint32_t)lane);
               const uint32_t rb = peer_addr(&tl->dbar[dp], (uint32_t)lane);
               const unsigned long long bits = __double_as_longlong(ss);
-              st_async_v4(ra, __uint_as_float((uint32_t)bits), __uint_as_float((uint32_t)(bits >> 32)),
-                          __int_as_float(ii), 0.f, rb);
+              st_async_v4(ra, __uint_as_float((uint32_t)bits),
+                          __uint_as_float((uint32_t)(bits >> 32)), __int_as_float(ii), 0.f, rb);
             }
           }
           if (!mbar_wait(&tl->dbar[dp], dph)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
-          double ss = lane < (int)C ? tl->drecv[dp][lane].s : -INFINITY;
-          int ii = lane < (int)C ? tl->drecv[dp][lane].idx : 0x7FFFFFFF;
+          double ss = lane < (int)J ? tl->drecv[dp][lane].s : -INFINITY;
+          int ii = lane < (int)J ? tl->drecv[dp][lane].idx : 0x7FFFFFFF;
           warp_c64(ss, ii);
           winner = ii;
           if (winner == 0x7FFFFFFF && mode == 1) {  // exact residual is zero everywhere
@@ -959,11 +993,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
         }
       } else {
         a.acc_len[unit] = acc_len;
-        for (int j = 0; j < a.R; ++j) {
+        for (int jj = 0; jj < a.R; ++jj) {
           int tok = -1;
-          if (j < acc_len) tok = a.draft[unit * a.K + j];
-          else if (j == acc_len) tok = emitted;
-          a.out_tokens[unit * a.R + j] = tok;
+          if (jj < acc_len) tok = a.draft[unit * a.K + jj];
+          else if (jj == acc_len) tok = emitted;
+          a.out_tokens[unit * a.R + jj] = tok;
         }
       }
     }
@@ -971,19 +1005,21 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
 
   // Last row's TV partials go to the leader, which hands them to its bookkeeping warp.
   if (want_tv && nrows > 0) {
-    bar_sync_n(ncomp);
-    if (warp == 0) {
-      float tvp = lane < nwarps ? tl->tvw[lane] : 0.f;
+    bar_sync_n(barid, gthr);
+    if (gwarp == 0) {
+      float tvp = lane < gnw ? gs->tvw[lane] : 0.f;
       tvp = warp_sum(tvp);
-      if (leader && lane == 0) mbar_arrive_expect_tx(&tl->fbar, C * 4u);
+      if (leader && grp == 0 && lane == 0) mbar_arrive_expect_tx(&tl->fbar, J * 4u);
       if (lane == 0)
-        st_async_b32(peer_addr(&tl->frecv[rank], 0), __float_as_uint(tvp), peer_addr(&tl->fbar, 0));
-      if (leader) {
+        st_async_b32(peer_addr(&tl->frecv[jslice], 0), __float_as_uint(tvp),
+                     peer_addr(&tl->fbar, 0));
+      if (leader && grp == 0) {
         if (!mbar_wait(&tl->fbar, 0)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
         const int slot = (int)(nrows % kLogN);
-        if (nrows >= kLogN && !mbar_wait(&tl->logempty[slot], (uint32_t)(((nrows / kLogN) - 1) & 1)))
+        if (nrows >= kLogN &&
+            !mbar_wait(&tl->logempty[slot], (uint32_t)(((nrows / kLogN) - 1) & 1)))
           raise_err(a.dev_err, SD_DEV_TIMEOUT);
-        if (lane < (int)C) tl->log[slot].m[lane].tvprev = tl->frecv[lane];
+        if (lane < (int)J) tl->log[slot].m[lane].tvprev = tl->frecv[lane];
         __syncwarp();
         if (lane == 0) mbar_arrive(&tl->logfull[slot]);
       }
@@ -994,7 +1030,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
 
 // ------------------------------------------------------------------ host side
 struct LaunchPlan {
-  int C, threads, stages, slice;
+  int C, groups, threads, stages, slice;
   uint32_t stage_bytes;
   size_t smem;
   int clusters_max;
@@ -1027,9 +1063,12 @@ static int max_active_clusters(const void* fn, int C, int threads, size_t smem) 
   return n;
 }
 
-// Chooses the cluster size C that keeps the most SMs busy for this many units:
-// each CTA must hold its slice in 32 registers per thread (<= 512 threads) and
-// at least two ring stages must fit in shared memory.  Plans are cached per
+// Chooses (cluster size C, warp groups per CTA) for this vocabulary: each
+// group holds its slice in 32 registers per thread per row, all groups plus the
+// service warp fit in 512 threads, J = C * groups <= 32 slices, and at least two
+// ring stages fit in shared memory.  Among the feasible choices it keeps the
+// most SMs busy for this many units, then prefers more groups (more overlap).
+// SMCSD_GROUPS=1..3 caps the number of groups.  Plans are cached per
 // (kernel, device, V, element size, unit count clipped at 4096).
 static bool make_plan(const void* fn, int V, int esize, int64_t units, LaunchPlan& best) {
   static std::mutex mu;
@@ -1044,32 +1083,40 @@ static bool make_plan(const void* fn, int V, int esize, int64_t units, LaunchPla
     best = hit->second;
     return true;
   }
+  int max_groups = kMaxGroups;
+  if (const char* env = getenv("SMCSD_GROUPS")) {
+    const int g = atoi(env);
+    if (g >= 1 && g <= kMaxGroups) max_groups = g;
+  }
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const size_t tail = sizeof(Tail) + 128;
   bool found = false;
   int64_t best_score = -1;
   for (int C = 1; C <= kMaxCluster; ++C) {
-    const int slice = (int)(((int64_t)(V + C - 1) / C + 7) / 8 * 8);
-    const int compute = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
-    const int threads = compute + 32;  // + the bookkeeping warp
-    if (threads > kMaxThreads) continue;
-    const uint32_t sb = (uint32_t)(((int64_t)slice * esize + 127) / 128 * 128);
-    int stages = 0;
-    for (int s = 4; s >= 2; --s)
-      if ((size_t)s * 2 * sb + tail <= (size_t)optin) {
-        stages = s;
-        break;
+    for (int ng = max_groups; ng >= 1; --ng) {
+      if (C * ng > kMaxSlices) continue;
+      const int slice = (int)(((int64_t)(V + C * ng - 1) / (C * ng) + 7) / 8 * 8);
+      const int gthr = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
+      const int threads = ng * gthr + 32;  // + the service warp
+      if (threads > kMaxThreads || gthr / 32 > kMaxWarps) continue;
+      const uint32_t sb = (uint32_t)(((int64_t)slice * ng * esize + 127) / 128 * 128);
+      int stages = 0;
+      for (int st = 4; st >= 2; --st)
+        if ((size_t)st * 2 * sb + tail <= (size_t)optin) {
+          stages = st;
+          break;
+        }
+      if (stages == 0) continue;
+      const size_t smem = (size_t)stages * 2 * sb + tail;
+      const int nc = max_active_clusters(fn, C, threads, smem);
+      if (nc <= 0) continue;
+      const int64_t score = (std::min<int64_t>(ukey, nc) * C) * 8 + ng;
+      if (score > best_score) {
+        best_score = score;
+        best = LaunchPlan{C, ng, threads, stages, slice, sb, smem, nc};
+        found = true;
       }
-    if (stages == 0) continue;
-    const size_t smem = (size_t)stages * 2 * sb + tail;
-    const int nc = max_active_clusters(fn, C, threads, smem);
-    if (nc <= 0) continue;
-    const int64_t score = std::min<int64_t>(ukey, nc) * C;
-    if (score > best_score) {
-      best_score = score;
-      best = LaunchPlan{C, threads, stages, slice, sb, smem, nc};
-      found = true;
     }
   }
   if (found) {
@@ -1085,6 +1132,7 @@ static sd_status launch_score(ScoreArgs& a, cudaStream_t stream) {
   LaunchPlan p;
   if (!make_plan(fn, a.V, (int)sizeof(TIn), a.units, p)) return SD_ERR_UNSUPPORTED;
   a.slice = p.slice;
+  a.groups = p.groups;
   a.stages = p.stages;
   a.stage_bytes = p.stage_bytes;
   const bool aligned = ((uintptr_t)a.zT % 16 == 0) && ((uintptr_t)a.zD % 16 == 0) &&

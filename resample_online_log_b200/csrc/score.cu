@@ -1028,6 +1028,465 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
   cluster_sync();  // all messages into this CTA have landed; peers may exit
 }
 
+// ====================================================================== SMC-SD kernel
+// Software-pipelined variant for SMC-SD rounds (every row has a target and a
+// draft half, the last row of each particle draws the bonus token).
+//
+// Iteration r of a CTA:
+//   1. move row r's slices from the ring to registers, per-thread and warp max;
+//   2. wait for row r-1's messages (sent one iteration ago, so their latency is
+//      hidden behind step 1), rebuild row r-1's normalisers, screen row r-1's
+//      bonus candidates if it ends a particle;
+//   3. one fused loop over this thread's entries: row r's exp2 (MUFU) and sums,
+//      row r-1's TV from its target exps (shared-memory buffer) and draft exps
+//      (registers) -- each slot is read and then overwritten in place;
+//   4. one CTA barrier; warp 0 combines the warp partials and pushes row r's
+//      message (carrying row r-1's TV partial) to every CTA of the cluster, and
+//      row r-1's bonus candidate to the leader.
+// Row r's exps thus stay on chip until its TV is taken one iteration later;
+// the bookkeeping warp of the leader turns the messages into log-weights, TV
+// and bonus tokens (deciding near-ties exactly in fp64).
+
+constexpr int kRing = 4;  // message slots: the bookkeeping warp may lag two rows
+
+struct alignas(128) SmcTail {
+  uint64_t full[2];
+  uint64_t rbar[kRing], cbar[kRing], bdone[kRing];
+  uint64_t fbar, pad;
+  Msg recv[kRing][kMaxCluster];
+  Cand crecv[kRing][kMaxCluster];
+  float frecv[kMaxCluster];
+  float4 wpart[2][kMaxWarps];  // warp scratch, by iteration parity: warps may run one
+  float tvw[2][kMaxWarps];     // iteration ahead of warp 0, which reads the previous one
+  Cand wcand[2][kMaxWarps];
+  float zx[2][2];
+};
+
+// fp64 lse of a row from per-slice partials (one per lane, `has` marks valid
+// lanes); the slice factors use MUFU exp2, the sum and the log are fp64.
+__device__ __noinline__ double row_lse_fast(float m, float s, float M, bool has, double tau64,
+                                            float cT) {
+  const double t = (has && m > -INFINITY) ? (double)s * (double)ex2((m - M) * cT) : 0.0;
+  return (double)M / tau64 + log(warp_sum_d(t));
+}
+
+// Exact fp64 bonus draw over a whole target row (a near-tie the fp32 screen
+// could not settle; rare).  One warp.
+template <typename TIn>
+__device__ __noinline__ int exact_bonus_row(const TIn* row, int V, double tau64, float inv_tau,
+                                            float lo_star, const Stream st, uint32_t rowid) {
+  const int lane = threadIdx.x & 31;
+  double best = -INFINITY;
+  int bi = 0x7FFFFFFF;
+  for (int q = lane; q * 4 < V; q += 32) {
+    const U4 w = st.at((uint32_t)q, rowid);
+    for (int j = 0; j < 4; ++j) {
+      const int v = q * 4 + j;
+      if (v >= V) break;
+      const float z = Elem<TIn>::get(row, v);
+      const float a32 = z * inv_tau;
+      if (!(a32 + kGumbelMaxF + 1e-3f >= lo_star)) continue;
+      const float g32 = gumbel_f32(uniform_f32(word_of(w, j)));
+      const float hi = a32 + g32 + 4e-6f + 4.8e-7f * (fabsf(a32) + 2.f * fabsf(g32));
+      if (!(hi >= lo_star)) continue;
+      const double s64 = (double)z / tau64 + gumbel_f64(uniform_f64(word_of(w, j)));
+      c64_merge(best, bi, s64, v);
+    }
+  }
+  warp_c64(best, bi);
+  return bi == 0x7FFFFFFF ? -1 : bi;
+}
+
+template <typename TIn>
+__device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32_t cid, uint32_t G,
+                             int64_t nrows, bool want_tv) {
+  const int lane = threadIdx.x & 31;
+  double logw_acc = 0.0;
+  bool unit_bad = false;
+  bool prev_bad = false;
+  int cuse[kRing] = {0, 0, 0, 0};
+  const Stream bst(a.seed, a.round, SD_STREAM_BONUS);
+  for (int64_t it = 0; it < nrows; ++it) {
+    const int slot = (int)(it % kRing);
+    const int64_t unit = cid + (it / a.R) * G;
+    const int k = (int)(it % a.R);
+    const int64_t rowT = unit * a.R + k;
+    if (!mbar_wait(&tl->rbar[slot], (uint32_t)((it / kRing) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+    const Msg* e = tl->recv[slot];
+    const bool has = lane < (int)C;
+    const float pm1 = has ? e[lane].mT : -INFINITY, ps1 = has ? e[lane].sT : 0.f;
+    const float pm2 = has ? e[lane].mD : -INFINITY, ps2 = has ? e[lane].sD : 0.f;
+    const float tvp = has ? e[lane].tvprev : 0.f;
+    const float MT = warp_max(pm1), MD = warp_max(pm2);
+    const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
+    const float SD = warp_sum(part_term(pm2, ps2, MD, a.cT));
+    const float tvsum = warp_sum(tvp);
+    const bool badT = !(MT > -INFINITY && MT < INFINITY && ST > 0.f && ST < INFINITY);
+    const bool badD = !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
+    const bool bad = badT || badD;
+    const double lse64T = row_lse_fast(pm1, ps1, MT, has, a.tau64, a.cT);
+    const double lse64D = row_lse_fast(pm2, ps2, MD, has, a.tau64, a.cT);
+    int x = -1;
+    float zxT = 0.f, zxD = 0.f;
+    if (k < a.K) {
+      x = a.draft[unit * a.K + k];
+      if (x >= 0 && x < a.V) {
+        const Msg& o = e[x / a.slice];
+        zxT = o.zxT;
+        zxD = o.zxD;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tl->bdone[slot]);  // message slot no longer needed
+    if (lane == 0) {
+      if (k == 0) {
+        logw_acc = 0.0;
+        unit_bad = false;
+      }
+      if (it > 0 && want_tv) {
+        const int64_t pu = cid + ((it - 1) / a.R) * G;
+        a.tv_out[pu * a.R + (int)((it - 1) % a.R)] = prev_bad ? NAN : 0.5f * tvsum;
+      }
+      if (bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
+      if (a.lse_out) {
+        a.lse_out[rowT * 2 + 0] = badT ? NAN : lse64T;
+        a.lse_out[rowT * 2 + 1] = badD ? NAN : lse64D;
+      }
+      if (k < a.K) {
+        const bool x_ok = x >= 0 && x < a.V;
+        double lp = NAN, lq = NAN;
+        if (!x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
+        if (x_ok && !bad) {
+          lp = (double)zxT / a.tau64 - lse64T;
+          lq = (double)zxD / a.tau64 - lse64D;
+        } else {
+          unit_bad = true;
+        }
+        logw_acc += lp - lq;
+        if (a.lp_out) {
+          a.lp_out[(unit * a.K + k) * 2 + 0] = lp;
+          a.lp_out[(unit * a.K + k) * 2 + 1] = lq;
+        }
+      } else {
+        const double prev = a.logw_prev ? a.logw_prev[unit] : 0.0;
+        a.logw_out[unit] = unit_bad ? NAN : prev + logw_acc;
+        if (a.tokens_out)
+          for (int jj = 0; jj < a.K; ++jj) a.tokens_out[unit * a.R + jj] = a.draft[unit * a.K + jj];
+      }
+    }
+    prev_bad = bad;
+    if (k == a.K) {  // bonus token: merge the slices' candidates
+      const uint32_t ph = (uint32_t)(cuse[slot] & 1);
+      ++cuse[slot];
+      if (!mbar_wait(&tl->cbar[slot], ph)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+      Cand c = has ? tl->crecv[slot][lane] : cand_empty();
+      c = warp_cand(c);
+      int winner;
+      if (badT || c.idx == 0x7FFFFFFF) winner = -1;
+      else if (c.ohi < c.lo) winner = c.idx;
+      else
+        winner = exact_bonus_row<TIn>((const TIn*)a.zT + rowT * a.ld, a.V, a.tau64, a.inv_tau, c.lo,
+                                      bst, (uint32_t)unit);
+      __syncwarp();
+      if (lane == 0) {
+        a.bonus_out[unit] = winner;
+        if (a.tokens_out) a.tokens_out[unit * a.R + a.K] = winner;
+      }
+    }
+  }
+  if (want_tv && nrows > 0) {  // the last row's TV arrives on its own
+    if (!mbar_wait(&tl->fbar, 0)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+    float v = lane < (int)C ? tl->frecv[lane] : 0.f;
+    v = warp_sum(v);
+    if (lane == 0) {
+      const int64_t pu = cid + ((nrows - 1) / a.R) * G;
+      a.tv_out[pu * a.R + (int)((nrows - 1) % a.R)] = prev_bad ? NAN : 0.5f * v;
+    }
+  }
+}
+
+// Fused per-thread pass: row r's exps (CUR) and row r-1's TV (PREV).
+template <int CPT, int EPC, bool CUR, bool PREV>
+__device__ __forceinline__ void fused_pass(float* xt, float* xd, float* dp, float4* tb, int tid,
+                                           int nthr, float mwT, float mwD, float cT, float scT,
+                                           float scD, float& sT, float& sD, float& tv) {
+  constexpr int EPT = CPT * EPC;
+  float2 aT = make_float2(0.f, 0.f), aD = make_float2(0.f, 0.f);
+  float t0 = 0.f, t1 = 0.f;
+  const float2 mT2 = make_float2(-mwT, -mwT), mD2 = make_float2(-mwD, -mwD);
+  const float2 c2 = make_float2(cT, cT);
+  const float2 sc2T = make_float2(scT, scT), sc2D = make_float2(scD, scD);
+#pragma unroll
+  for (int q = 0; q < EPT / 4; ++q) {
+    float4& slot = tb[q * nthr + tid];
+    float4 old = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (PREV) old = slot;
+    float4 nw;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = q * 4 + h * 2;
+      if (PREV) {
+        const float2 ot = h == 0 ? make_float2(old.x, old.y) : make_float2(old.z, old.w);
+        const float2 p = __fmul2_rn(ot, sc2T);
+        const float2 qq = __fmul2_rn(make_float2(dp[i], dp[i + 1]), sc2D);
+        const float2 d = __fadd2_rn(p, make_float2(-qq.x, -qq.y));
+        t0 += fabsf(d.x);
+        t1 += fabsf(d.y);
+      }
+      if (CUR) {
+        const float2 at = __fmul2_rn(__fadd2_rn(make_float2(xt[i], xt[i + 1]), mT2), c2);
+        const float2 ad = __fmul2_rn(__fadd2_rn(make_float2(xd[i], xd[i + 1]), mD2), c2);
+        const float2 et = make_float2(ex2(at.x), ex2(at.y));
+        const float2 ed = make_float2(ex2(ad.x), ex2(ad.y));
+        aT = __fadd2_rn(aT, et);
+        aD = __fadd2_rn(aD, ed);
+        if (h == 0) {
+          nw.x = et.x;
+          nw.y = et.y;
+        } else {
+          nw.z = et.x;
+          nw.w = et.y;
+        }
+        dp[i] = ed.x;
+        dp[i + 1] = ed.y;
+      }
+    }
+    if (CUR) slot = nw;
+  }
+  sT = aT.x + aT.y;
+  sD = aD.x + aD.y;
+  tv = t0 + t1;
+  (void)EPC;
+}
+
+template <typename TIn, int CPT>
+__global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) {
+  constexpr int EPC = 16 / (int)sizeof(TIn);
+  constexpr int EPT = CPT * EPC;
+  static_assert(EPT == kEPT, "entries per thread");
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ncomp = blockDim.x - 32, nwarps = ncomp >> 5;  // last warp: bookkeeping
+  const uint32_t rank = cluster_rank(), C = cluster_size();
+  const uint32_t cid = cluster_id(), G = num_clusters();
+  float4* tbuf = reinterpret_cast<float4*>(smem + (size_t)2 * 2 * a.stage_bytes);
+  SmcTail* tl = reinterpret_cast<SmcTail*>(smem + (size_t)2 * 2 * a.stage_bytes +
+                                           (size_t)ncomp * EPT * sizeof(float));
+
+  const int s0 = (int)rank * a.slice;
+  const int len = max(0, min(a.slice, a.V - s0));
+  const int tma_len = a.use_tma ? ((len * (int)sizeof(TIn)) & ~15) / (int)sizeof(TIn) : 0;
+  const uint32_t tma_bytes = (uint32_t)tma_len * (uint32_t)sizeof(TIn);
+  const int64_t my_units = (int64_t)cid < a.units ? (a.units - 1 - cid) / G + 1 : 0;
+  const int64_t nrows = my_units * a.R;
+  const bool leader = rank == 0;
+  const bool want_tv = a.tv_out != nullptr;
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) mbar_init(&tl->full[s], 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&tl->rbar[i], 1);
+      mbar_init(&tl->cbar[i], 1);
+      mbar_init(&tl->bdone[i], 1);
+    }
+    mbar_init(&tl->fbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  cluster_sync();
+
+  if (warp == nwarps) {
+    if (leader) smc_bookkeep<TIn>(a, tl, C, cid, G, nrows, want_tv);
+    cluster_sync();
+    return;
+  }
+
+  const uint64_t pol = policy_evict_first();
+  auto issue = [&](int64_t it) {
+    const int s = (int)(it & 1);
+    const int64_t unit = cid + (it / a.R) * G;
+    const int64_t row = unit * a.R + (int)(it % a.R);
+    unsigned char* stg = smem + (size_t)s * 2 * a.stage_bytes;
+    mbar_arrive_expect_tx(&tl->full[s], tma_bytes * 2u);
+    if (tma_bytes) {
+      bulk_load(stg, (const TIn*)a.zT + row * a.ld + s0, tma_bytes, &tl->full[s], pol);
+      bulk_load(stg + a.stage_bytes, (const TIn*)a.zD + row * a.ld + s0, tma_bytes, &tl->full[s], pol);
+    }
+  };
+  if (tid == 0)
+    for (int64_t it = 0; it < nrows && it < 2; ++it) issue(it);
+
+  float xt[EPT], xd[EPT], dp[EPT];
+  float mwT_p = 0.f, mwD_p = 0.f;  // previous row's warp maxima (safe forms)
+  bool okT_p = false, okD_p = false;  // ... and whether they were finite
+  bool prev_valid = false;
+  const float inv_tau = a.inv_tau;
+
+  for (int64_t it = 0; it <= nrows; ++it) {
+    const bool cur = it < nrows;
+    const int64_t unit = cid + (it / a.R) * G;
+    const int k = (int)(it % a.R);
+    const int64_t row = unit * a.R + k;
+    float mwT = -INFINITY, mwD = -INFINITY;
+    bool owner = false;
+    int par = (int)(it & 1);
+    if (cur) {
+      if (!mbar_wait(&tl->full[par], (uint32_t)((it >> 1) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+      const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes);
+      const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes + a.stage_bytes);
+      const TIn* gT = (const TIn*)a.zT + row * a.ld + s0;
+      const TIn* gD = (const TIn*)a.zD + row * a.ld + s0;
+      const float mt = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, tid, ncomp);
+      const float md = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, tid, ncomp);
+      if (k < a.K) {
+        const int x = a.draft[unit * a.K + k];
+        owner = x >= s0 && x < s0 + len;
+        if (owner) {
+          const int le = x - s0;
+          if (((le / EPC) % ncomp) == tid) {
+            tl->zx[par][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
+            tl->zx[par][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
+          }
+        }
+      }
+      mwT = warp_max(mt);
+      mwD = warp_max(md);
+    }
+    const float mwTs = mwT == -INFINITY ? 0.f : mwT;
+    const float mwDs = mwD == -INFINITY ? 0.f : mwD;
+
+    // ---- previous row: normalisers, bonus screen ----
+    float scT = 0.f, scD = 0.f;
+    bool prev_bonus = false;
+    if (prev_valid) {
+      const int64_t pit = it - 1;
+      const int pslot = (int)(pit % kRing);
+      const int pk = (int)(pit % a.R);
+      const int64_t punit = cid + (pit / a.R) * G;
+      if (!mbar_wait(&tl->rbar[pslot], (uint32_t)((pit / kRing) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+      const Msg* rv = tl->recv[pslot];
+      const bool has = lane < (int)C;
+      const float pm1 = has ? rv[lane].mT : -INFINITY, ps1 = has ? rv[lane].sT : 0.f;
+      const float pm2 = has ? rv[lane].mD : -INFINITY, ps2 = has ? rv[lane].sD : 0.f;
+      const float MT = warp_max(pm1), MD = warp_max(pm2);
+      const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
+      const float SD = warp_sum(part_term(pm2, ps2, MD, a.cT));
+      const bool badT = !(MT > -INFINITY && MT < INFINITY && ST > 0.f && ST < INFINITY);
+      const bool badD = !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
+      scT = (!badT && okT_p) ? ex2((mwT_p - MT) * a.cT) / ST : 0.f;
+      scD = (!badD && okD_p) ? ex2((mwD_p - MD) * a.cT) / SD : 0.f;
+      if (pk == a.K) {
+        prev_bonus = true;
+        Cand cd = cand_empty();
+        if (!badT && okT_p) {
+          // Tref = M/tau + g_min - margin: a lower bound on the winning score.
+          const float margin = 1e-5f + 2e-7f * fabsf(MT * inv_tau);
+          const float rho = ex2((mwT_p - MT) * a.cT + (-kGumbelMinF + margin) * kLog2e);
+          const Stream st(a.seed, a.round, SD_STREAM_BONUS);
+#pragma unroll
+          for (int q = 0; q < EPT / 4; ++q) {
+            const int c = q / (EPC / 4);
+            const int e0 = (tid + c * ncomp) * EPC + (q % (EPC / 4)) * 4;
+            if (e0 >= len) continue;
+            const float4 ev = tbuf[q * ncomp + tid];
+            const float y0 = ev.x * rho, y1 = ev.y * rho, y2 = ev.z * rho, y3 = ev.w * rho;
+            if (fmaxf(fmaxf(y0, y1), fmaxf(y2, y3)) < kYSkip) continue;
+            const int v0 = s0 + e0;
+            const U4 w = st.at((uint32_t)(v0 >> 2), (uint32_t)punit);
+            const float u0 = uniform_f32(w.x), u1 = uniform_f32(w.y);
+            const float u2 = uniform_f32(w.z), u3 = uniform_f32(w.w);
+            const bool k0 = keep_bonus(y0, u0) && e0 + 0 < len;
+            const bool k1 = keep_bonus(y1, u1) && e0 + 1 < len;
+            const bool k2 = keep_bonus(y2, u2) && e0 + 2 < len;
+            const bool k3 = keep_bonus(y3, u3) && e0 + 3 < len;
+            const float mw_a = mwT_p * inv_tau;
+            if (k0 | k1 | k2 | k3) {
+              if (k0) cd = cand_merge(cd, bonus_cand(ev.x, u0, mw_a, v0));
+              if (k1) cd = cand_merge(cd, bonus_cand(ev.y, u1, mw_a, v0 + 1));
+              if (k2) cd = cand_merge(cd, bonus_cand(ev.z, u2, mw_a, v0 + 2));
+              if (k3) cd = cand_merge(cd, bonus_cand(ev.w, u3, mw_a, v0 + 3));
+            }
+          }
+        }
+        cd = warp_cand(cd);
+        if (lane == 0) tl->wcand[par][warp] = cd;
+        (void)punit;
+      }
+    }
+
+    // ---- fused pass: row r exps + row r-1 TV ----
+    float sT = 0.f, sD = 0.f, tv = 0.f;
+    if (cur && prev_valid)
+      fused_pass<CPT, EPC, true, true>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD, sT,
+                                       sD, tv);
+    else if (cur)
+      fused_pass<CPT, EPC, true, false>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD,
+                                        sT, sD, tv);
+    else
+      fused_pass<CPT, EPC, false, true>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD,
+                                        sT, sD, tv);
+    sT = warp_sum(sT);
+    sD = warp_sum(sD);
+    tv = warp_sum(tv);
+    if (lane == 0) {
+      tl->wpart[par][warp] = make_float4(mwT, sT, mwD, sD);
+      tl->tvw[par][warp] = tv;
+    }
+    bar_sync_n(1, ncomp);  // (A) warp partials visible; this row's stage is free
+    if (cur && tid == 0 && it + 2 < nrows) issue(it + 2);
+    if (warp == 0) {
+      const float tvp = lane < nwarps ? tl->tvw[par][lane] : 0.f;
+      const float tvc = want_tv ? warp_sum(tvp) : 0.f;
+      if (cur) {
+        const float4 wp =
+            lane < nwarps ? tl->wpart[par][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        Msg m;
+        m.mT = warp_max(wp.x);
+        m.mD = warp_max(wp.z);
+        m.sT = warp_sum(part_term(wp.x, wp.y, m.mT, a.cT));
+        m.sD = warp_sum(part_term(wp.z, wp.w, m.mD, a.cT));
+        m.tvprev = tvc;
+        m.aux = 0;
+        m.zxT = owner ? tl->zx[par][0] : 0.f;
+        m.zxD = owner ? tl->zx[par][1] : 0.f;
+        const int slot = (int)(it % kRing);
+        if (leader && it >= 2 && !mbar_wait(&tl->bdone[(it - 2) % kRing], (uint32_t)(((it - 2) / kRing) & 1)))
+          raise_err(a.dev_err, SD_DEV_TIMEOUT);
+        if (lane == 0) mbar_arrive_expect_tx(&tl->rbar[slot], C * (uint32_t)sizeof(Msg));
+        if (lane < (int)C) {
+          const uint32_t ra = peer_addr(&tl->recv[slot][rank], (uint32_t)lane);
+          const uint32_t rb = peer_addr(&tl->rbar[slot], (uint32_t)lane);
+          st_async_v4(ra, m.mT, m.sT, m.mD, m.sD, rb);
+          st_async_v4(ra + 16, m.zxT, m.zxD, m.tvprev, 0.f, rb);
+        }
+      } else if (want_tv && prev_valid) {  // final iteration: the last row's TV goes to the leader
+        if (leader && lane == 0) mbar_arrive_expect_tx(&tl->fbar, C * 4u);
+        if (lane == 0)
+          st_async_b32(peer_addr(&tl->frecv[rank], 0), __float_as_uint(tvc), peer_addr(&tl->fbar, 0));
+      }
+      if (prev_bonus) {  // row r-1's bonus candidate goes to the leader
+        const int pslot = (int)((it - 1) % kRing);
+        Cand c2 = lane < nwarps ? tl->wcand[par][lane] : cand_empty();
+        c2 = warp_cand(c2);
+        if (leader && lane == 0) mbar_arrive_expect_tx(&tl->cbar[pslot], C * (uint32_t)sizeof(Cand));
+        if (lane == 0) {
+          const uint32_t ra = peer_addr(&tl->crecv[pslot][rank], 0);
+          const uint32_t rb = peer_addr(&tl->cbar[pslot], 0);
+          st_async_v4(ra, c2.s, c2.lo, c2.hi, c2.ohi, rb);
+          st_async_v4(ra + 16, __int_as_float(c2.idx), 0.f, 0.f, 0.f, rb);
+        }
+      }
+    }
+    mwT_p = mwTs;
+    mwD_p = mwDs;
+    okT_p = mwT > -INFINITY;
+    okD_p = mwD > -INFINITY;
+    prev_valid = cur;
+  }
+  cluster_sync();
+}
+
 // ------------------------------------------------------------------ host side
 struct LaunchPlan {
   int C, groups, threads, stages, slice;
@@ -1126,6 +1585,87 @@ static bool make_plan(const void* fn, int V, int esize, int64_t units, LaunchPla
   return found;
 }
 
+// Launch plan of the pipelined SMC-SD kernel: one warp group per CTA, two
+// ring stages, plus the target-exps buffer (32 fp32 per compute thread).
+static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, LaunchPlan& best) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int, int, int64_t>, LaunchPlan> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t ukey = std::min<int64_t>(units, 4096);
+  const auto key = std::make_tuple(fn, dev, V, esize, ukey);
+  auto hit = cache.find(key);
+  if (hit != cache.end()) {
+    best = hit->second;
+    return true;
+  }
+  int optin = 0;
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  bool found = false;
+  int64_t best_score = -1;
+  for (int C = 1; C <= kMaxCluster; ++C) {
+    const int slice = (int)(((int64_t)(V + C - 1) / C + 7) / 8 * 8);
+    const int ncomp = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
+    const int threads = ncomp + 32;
+    if (threads > kMaxThreads || ncomp / 32 > kMaxWarps) continue;
+    const uint32_t sb = (uint32_t)(((int64_t)slice * esize + 127) / 128 * 128);
+    const size_t smem = (size_t)2 * 2 * sb + (size_t)ncomp * kEPT * 4 + sizeof(SmcTail) + 128;
+    if (smem > (size_t)optin) continue;
+    const int nc = max_active_clusters(fn, C, threads, smem);
+    if (nc <= 0) continue;
+    const int64_t score = std::min<int64_t>(ukey, nc) * C;
+    if (score > best_score) {
+      best_score = score;
+      best = LaunchPlan{C, 1, threads, 2, slice, sb, smem, nc};
+      found = true;
+    }
+  }
+  if (found) {
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)best.smem);
+    cache[key] = best;
+  }
+  return found;
+}
+
+template <typename TIn>
+static sd_status launch_smc(ScoreArgs& a, cudaStream_t stream) {
+  const void* fn = (const void*)smc_kernel<TIn, (int)(kEPT * sizeof(TIn) / 16)>;
+  LaunchPlan p;
+  if (!make_plan_smc(fn, a.V, (int)sizeof(TIn), a.units, p)) return SD_ERR_UNSUPPORTED;
+  a.slice = p.slice;
+  a.groups = 1;
+  a.stages = 2;
+  a.stage_bytes = p.stage_bytes;
+  const bool aligned = ((uintptr_t)a.zT % 16 == 0) && ((uintptr_t)a.zD % 16 == 0) &&
+                       ((a.ld * (int64_t)sizeof(TIn)) % 16 == 0);
+  a.use_tma = aligned ? 1 : 0;
+  const int64_t nclusters = std::min<int64_t>(a.units, p.clusters_max);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return SD_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nclusters * p.C));
+  cfg.blockDim = dim3(p.threads);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = p.C;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, smc_kernel<TIn, (int)(kEPT * sizeof(TIn) / 16)>, a);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SD_ERR_CUDA;
+  }
+  return SD_OK;
+}
+
 template <typename TIn, bool VERIFY>
 static sd_status launch_score(ScoreArgs& a, cudaStream_t stream) {
   const void* fn = kernel_ptr<TIn, VERIFY>();
@@ -1209,7 +1749,7 @@ extern "C" sd_status smcsd_score(const void* zT, const void* zD, sd_dtype dt, in
   a.lp_out = lp_out;
   a.dev_err = dev_err;
   cudaStream_t s = (cudaStream_t)stream;
-  return dt == SD_BF16 ? launch_score<uint16_t, false>(a, s) : launch_score<float, false>(a, s);
+  return dt == SD_BF16 ? launch_smc<uint16_t>(a, s) : launch_smc<float>(a, s);
 }
 
 extern "C" sd_status sd_verify_reject(const void* zT, const void* zD, sd_dtype dt, int B, int K,

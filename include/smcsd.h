@@ -187,7 +187,7 @@ SMCSD_API sd_status sd_verify_reject(const void* zT, const void* zD, sd_dtype dt
  * idx_out    device int32 [rows, k] (required).
  * score_out  device fp32 [rows, k]: s_v + g_v (or NULL).
  * logp_out   device fp32 [rows, k]: s_v - logsumexp(s) (or NULL).
- * Requirements: rows >= 0, 1 <= k <= 64, k <= V, ld >= V.
+ * Requirements: rows >= 0, 1 <= k <= 16, k <= V, ld >= V.
  * Faults: rows with NaN / +inf or all -inf -> SD_DEV_NONFINITE, ids -1;
  *   ranks with no finite entry left are -1.
  */
@@ -203,7 +203,7 @@ SMCSD_API sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, int
  * global ids.
  * idx   device int32 [rows, L];  prob device fp32 [rows, L];
  * idx_out device int32 [rows, k].
- * Requirements: rows >= 0, 1 <= L <= 64, 1 <= k <= L.
+ * Requirements: rows >= 0, 1 <= L <= 16, 1 <= k <= L.
  * Faults: NaN / negative / infinite probability -> SD_DEV_NONFINITE, ids -1.
  */
 SMCSD_API sd_status gumbel_topk_sparse(const int32_t* idx, const float* prob, int rows, int L, int k,

@@ -1062,6 +1062,36 @@ struct alignas(128) SmcTail {
   float zx[2][2];
 };
 
+// Paired warp reductions (two independent values per shuffle round).
+__device__ __forceinline__ void warp_max2(float& a, float& b) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float x = __shfl_xor_sync(0xffffffffu, a, o);
+    const float y = __shfl_xor_sync(0xffffffffu, b, o);
+    a = fmaxf(a, x);
+    b = fmaxf(b, y);
+  }
+}
+__device__ __forceinline__ void warp_sum2(float& a, float& b) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float x = __shfl_xor_sync(0xffffffffu, a, o);
+    const float y = __shfl_xor_sync(0xffffffffu, b, o);
+    a += x;
+    b += y;
+  }
+}
+__device__ __forceinline__ void warp_sum3(float& a, float& b, float& c) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float x = __shfl_xor_sync(0xffffffffu, a, o);
+    const float y = __shfl_xor_sync(0xffffffffu, b, o);
+    const float z = __shfl_xor_sync(0xffffffffu, c, o);
+    a += x;
+    b += y;
+    c += z;
+  }
+}
 // fp64 lse of a row from per-slice partials (one per lane, `has` marks valid
 // lanes); the slice factors use MUFU exp2, the sum and the log are fp64.
 __device__ __noinline__ double row_lse_fast(float m, float s, float M, bool has, double tau64,
@@ -1099,28 +1129,29 @@ __device__ __noinline__ int exact_bonus_row(const TIn* row, int V, double tau64,
 
 template <typename TIn>
 __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32_t cid, uint32_t G,
-                             int64_t nrows, bool want_tv) {
+                             int nrows, bool want_tv) {
   const int lane = threadIdx.x & 31;
   double logw_acc = 0.0;
   bool unit_bad = false;
   bool prev_bad = false;
   int cuse[kRing] = {0, 0, 0, 0};
   const Stream bst(a.seed, a.round, SD_STREAM_BONUS);
-  for (int64_t it = 0; it < nrows; ++it) {
-    const int slot = (int)(it % kRing);
-    const int64_t unit = cid + (it / a.R) * G;
-    const int k = (int)(it % a.R);
+  int k = 0;
+  int64_t unit = cid;
+  int64_t prev_row = -1;
+  for (int it = 0; it < nrows; ++it, prev_row = unit * a.R + k, (++k == a.R ? (k = 0, unit += G) : 0)) {
+    const int slot = it % kRing;
     const int64_t rowT = unit * a.R + k;
     if (!mbar_wait(&tl->rbar[slot], (uint32_t)((it / kRing) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
     const Msg* e = tl->recv[slot];
     const bool has = lane < (int)C;
     const float pm1 = has ? e[lane].mT : -INFINITY, ps1 = has ? e[lane].sT : 0.f;
     const float pm2 = has ? e[lane].mD : -INFINITY, ps2 = has ? e[lane].sD : 0.f;
-    const float tvp = has ? e[lane].tvprev : 0.f;
-    const float MT = warp_max(pm1), MD = warp_max(pm2);
-    const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
-    const float SD = warp_sum(part_term(pm2, ps2, MD, a.cT));
-    const float tvsum = warp_sum(tvp);
+    float tvsum = has ? e[lane].tvprev : 0.f;
+    float MT = pm1, MD = pm2;
+    warp_max2(MT, MD);
+    float ST = part_term(pm1, ps1, MT, a.cT), SD = part_term(pm2, ps2, MD, a.cT);
+    warp_sum3(ST, SD, tvsum);
     const bool badT = !(MT > -INFINITY && MT < INFINITY && ST > 0.f && ST < INFINITY);
     const bool badD = !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
     const bool bad = badT || badD;
@@ -1143,10 +1174,7 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
         logw_acc = 0.0;
         unit_bad = false;
       }
-      if (it > 0 && want_tv) {
-        const int64_t pu = cid + ((it - 1) / a.R) * G;
-        a.tv_out[pu * a.R + (int)((it - 1) % a.R)] = prev_bad ? NAN : 0.5f * tvsum;
-      }
+      if (it > 0 && want_tv) a.tv_out[prev_row] = prev_bad ? NAN : 0.5f * tvsum;
       if (bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
       if (a.lse_out) {
         a.lse_out[rowT * 2 + 0] = badT ? NAN : lse64T;
@@ -1198,10 +1226,7 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
     if (!mbar_wait(&tl->fbar, 0)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
     float v = lane < (int)C ? tl->frecv[lane] : 0.f;
     v = warp_sum(v);
-    if (lane == 0) {
-      const int64_t pu = cid + ((nrows - 1) / a.R) * G;
-      a.tv_out[pu * a.R + (int)((nrows - 1) % a.R)] = prev_bad ? NAN : 0.5f * v;
-    }
+    if (lane == 0) a.tv_out[prev_row] = prev_bad ? NAN : 0.5f * v;
   }
 }
 
@@ -1215,7 +1240,6 @@ __device__ __forceinline__ void fused_pass(float* xt, float* xd, float* dp, floa
   float t0 = 0.f, t1 = 0.f;
   const float2 mT2 = make_float2(-mwT, -mwT), mD2 = make_float2(-mwD, -mwD);
   const float2 c2 = make_float2(cT, cT);
-  const float2 sc2T = make_float2(scT, scT), sc2D = make_float2(scD, scD);
 #pragma unroll
   for (int q = 0; q < EPT / 4; ++q) {
     float4& slot = tb[q * nthr + tid];
@@ -1225,13 +1249,10 @@ __device__ __forceinline__ void fused_pass(float* xt, float* xd, float* dp, floa
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int i = q * 4 + h * 2;
-      if (PREV) {
-        const float2 ot = h == 0 ? make_float2(old.x, old.y) : make_float2(old.z, old.w);
-        const float2 p = __fmul2_rn(ot, sc2T);
-        const float2 qq = __fmul2_rn(make_float2(dp[i], dp[i + 1]), sc2D);
-        const float2 d = __fadd2_rn(p, make_float2(-qq.x, -qq.y));
-        t0 += fabsf(d.x);
-        t1 += fabsf(d.y);
+      if (PREV) {  // separately rounded products: identical rows give exactly 0
+        const float o0 = h == 0 ? old.x : old.z, o1 = h == 0 ? old.y : old.w;
+        t0 += fabsf(__fmul_rn(o0, scT) - __fmul_rn(dp[i], scD));
+        t1 += fabsf(__fmul_rn(o1, scT) - __fmul_rn(dp[i + 1], scD));
       }
       if (CUR) {
         const float2 at = __fmul2_rn(__fadd2_rn(make_float2(xt[i], xt[i + 1]), mT2), c2);
@@ -1259,6 +1280,24 @@ __device__ __forceinline__ void fused_pass(float* xt, float* xd, float* dp, floa
   (void)EPC;
 }
 
+// Row normalisers from per-slice (max, sum) partials held one per lane.
+struct Norm {
+  float MT, ST, MD, SD;
+  bool badT, badD;
+};
+__device__ __forceinline__ Norm row_norm(float pm1, float ps1, float pm2, float ps2, float cT) {
+  Norm n;
+  n.MT = pm1;
+  n.MD = pm2;
+  warp_max2(n.MT, n.MD);
+  n.ST = part_term(pm1, ps1, n.MT, cT);
+  n.SD = part_term(pm2, ps2, n.MD, cT);
+  warp_sum2(n.ST, n.SD);
+  n.badT = !(n.MT > -INFINITY && n.MT < INFINITY && n.ST > 0.f && n.ST < INFINITY);
+  n.badD = !(n.MD > -INFINITY && n.MD < INFINITY && n.SD > 0.f && n.SD < INFINITY);
+  return n;
+}
+
 template <typename TIn, int CPT>
 __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) {
   constexpr int EPC = 16 / (int)sizeof(TIn);
@@ -1267,7 +1306,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ncomp = blockDim.x - 32, nwarps = ncomp >> 5;  // last warp: bookkeeping
+  // warps [0, nwarps): compute; warp nwarps: communication; warp nwarps+1: bookkeeping
+  const int ncomp = blockDim.x - 64, nwarps = ncomp >> 5;
   const uint32_t rank = cluster_rank(), C = cluster_size();
   const uint32_t cid = cluster_id(), G = num_clusters();
   float4* tbuf = reinterpret_cast<float4*>(smem + (size_t)2 * 2 * a.stage_bytes);
@@ -1279,7 +1319,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
   const int tma_len = a.use_tma ? ((len * (int)sizeof(TIn)) & ~15) / (int)sizeof(TIn) : 0;
   const uint32_t tma_bytes = (uint32_t)tma_len * (uint32_t)sizeof(TIn);
   const int64_t my_units = (int64_t)cid < a.units ? (a.units - 1 - cid) / G + 1 : 0;
-  const int64_t nrows = my_units * a.R;
+  const int nrows = (int)(my_units * a.R);
   const bool leader = rank == 0;
   const bool want_tv = a.tv_out != nullptr;
 
@@ -1296,17 +1336,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
   __syncthreads();
   cluster_sync();
 
-  if (warp == nwarps) {
+  if (warp == nwarps + 1) {  // ---------------- bookkeeping (leader only)
     if (leader) smc_bookkeep<TIn>(a, tl, C, cid, G, nrows, want_tv);
     cluster_sync();
     return;
   }
 
   const uint64_t pol = policy_evict_first();
-  auto issue = [&](int64_t it) {
-    const int s = (int)(it & 1);
-    const int64_t unit = cid + (it / a.R) * G;
-    const int64_t row = unit * a.R + (int)(it % a.R);
+  // stage (row & 1) <- row `it` of this cluster: unit cid + (it / R) * G, position it % R
+  auto issue = [&](int it) {
+    const int s = it & 1;
+    const int64_t row = ((int64_t)cid + (int64_t)(it / a.R) * G) * a.R + (it % a.R);
     unsigned char* stg = smem + (size_t)s * 2 * a.stage_bytes;
     mbar_arrive_expect_tx(&tl->full[s], tma_bytes * 2u);
     if (tma_bytes) {
@@ -1314,75 +1354,112 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
       bulk_load(stg + a.stage_bytes, (const TIn*)a.zD + row * a.ld + s0, tma_bytes, &tl->full[s], pol);
     }
   };
-  if (tid == 0)
-    for (int64_t it = 0; it < nrows && it < 2; ++it) issue(it);
 
-  float xt[EPT], xd[EPT], dp[EPT];
-  float mwT_p = 0.f, mwD_p = 0.f;  // previous row's warp maxima (safe forms)
-  bool okT_p = false, okD_p = false;  // ... and whether they were finite
-  bool prev_valid = false;
-  const float inv_tau = a.inv_tau;
-
-  for (int64_t it = 0; it <= nrows; ++it) {
-    const bool cur = it < nrows;
-    const int64_t unit = cid + (it / a.R) * G;
-    const int k = (int)(it % a.R);
-    const int64_t row = unit * a.R + k;
-    float mwT = -INFINITY, mwD = -INFINITY;
-    bool owner = false;
-    int par = (int)(it & 1);
-    if (cur) {
-      if (!mbar_wait(&tl->full[par], (uint32_t)((it >> 1) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
-      const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes);
-      const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes + a.stage_bytes);
-      const TIn* gT = (const TIn*)a.zT + row * a.ld + s0;
-      const TIn* gD = (const TIn*)a.zD + row * a.ld + s0;
-      const float mt = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, tid, ncomp);
-      const float md = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, tid, ncomp);
-      if (k < a.K) {
-        const int x = a.draft[unit * a.K + k];
-        owner = x >= s0 && x < s0 + len;
-        if (owner) {
-          const int le = x - s0;
-          if (((le / EPC) % ncomp) == tid) {
-            tl->zx[par][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
-            tl->zx[par][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
-          }
+  if (warp == nwarps) {  // ---------------- communication warp
+    if (lane == 0)
+      for (int it = 0; it < nrows && it < 2; ++it) issue(it);
+    int k = 0;
+    for (int it = 0; it <= nrows; ++it) {
+      const bool cur = it < nrows;
+      const int par = it & 1;
+      bar_sync_n(1, ncomp + 32);  // compute warps have posted their partials of iteration `it`
+      if (cur && lane == 0 && it + 2 < nrows) issue(it + 2);  // stage `par` is free again
+      float tvp = lane < nwarps ? tl->tvw[par][lane] : 0.f;
+      if (cur) {
+        const float4 wp =
+            lane < nwarps ? tl->wpart[par][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        float mT = wp.x, mD = wp.z;
+        warp_max2(mT, mD);
+        float sT = part_term(wp.x, wp.y, mT, a.cT), sD = part_term(wp.z, wp.w, mD, a.cT);
+        warp_sum3(sT, sD, tvp);
+        const bool owner_known = k < a.K;
+        float zxT = 0.f, zxD = 0.f;
+        if (owner_known) {
+          zxT = tl->zx[par][0];
+          zxD = tl->zx[par][1];
+        }
+        const int slot = it % kRing;
+        if (leader && it >= 2 &&
+            !mbar_wait(&tl->bdone[(it - 2) % kRing], (uint32_t)(((it - 2) / kRing) & 1)))
+          raise_err(a.dev_err, SD_DEV_TIMEOUT);
+        if (lane == 0) mbar_arrive_expect_tx(&tl->rbar[slot], C * (uint32_t)sizeof(Msg));
+        if (lane < (int)C) {
+          const uint32_t ra = peer_addr(&tl->recv[slot][rank], (uint32_t)lane);
+          const uint32_t rb = peer_addr(&tl->rbar[slot], (uint32_t)lane);
+          st_async_v4(ra, mT, sT, mD, sD, rb);
+          st_async_v4(ra + 16, zxT, zxD, want_tv ? tvp : 0.f, 0.f, rb);
+        }
+      } else {
+        tvp = warp_sum(tvp);
+        if (want_tv && nrows > 0) {  // final iteration: the last row's TV goes to the leader
+          if (leader && lane == 0) mbar_arrive_expect_tx(&tl->fbar, C * 4u);
+          if (lane == 0)
+            st_async_b32(peer_addr(&tl->frecv[rank], 0), __float_as_uint(tvp), peer_addr(&tl->fbar, 0));
         }
       }
-      mwT = warp_max(mt);
-      mwD = warp_max(md);
+      if (it > 0 && ((it - 1) % a.R) == a.K) {  // row it-1's bonus candidate goes to the leader
+        const int pslot = (it - 1) % kRing;
+        Cand c2 = lane < nwarps ? tl->wcand[par][lane] : cand_empty();
+        c2 = warp_cand(c2);
+        if (leader && lane == 0) mbar_arrive_expect_tx(&tl->cbar[pslot], C * (uint32_t)sizeof(Cand));
+        if (lane == 0) {
+          const uint32_t ra = peer_addr(&tl->crecv[pslot][rank], 0);
+          const uint32_t rb = peer_addr(&tl->cbar[pslot], 0);
+          st_async_v4(ra, c2.s, c2.lo, c2.hi, c2.ohi, rb);
+          st_async_v4(ra + 16, __int_as_float(c2.idx), 0.f, 0.f, 0.f, rb);
+        }
+      }
+      if (++k == a.R) k = 0;
     }
-    const float mwTs = mwT == -INFINITY ? 0.f : mwT;
-    const float mwDs = mwD == -INFINITY ? 0.f : mwD;
+    cluster_sync();
+    return;
+  }
 
-    // ---- previous row: normalisers, bonus screen ----
+  // ---------------- compute warps
+  float xt[EPT], xd[EPT], dp[EPT];
+  float mwT_p = 0.f, mwD_p = 0.f;  // previous row's warp maxima (safe forms)
+  bool okT_p = false, okD_p = false;
+  const float inv_tau = a.inv_tau;
+  int k = 0;          // position of row `it` within its particle
+  int64_t unit = cid; // particle of row `it`
+  int x_next = (nrows > 0 && a.K > 0) ? a.draft[(int64_t)cid * a.K] : -1;
+
+  for (int it = 0; it <= nrows; ++it) {
+    const bool cur = it < nrows;
+    const bool prev = it > 0;
+    const int par = it & 1;
+    const int x = (cur && k < a.K) ? x_next : -1;
+    {  // prefetch the draft token of row it+1
+      int kn = k + 1;
+      int64_t un = unit;
+      if (kn == a.R) {
+        kn = 0;
+        un += G;
+      }
+      x_next = (it + 1 < nrows && kn < a.K) ? a.draft[un * a.K + kn] : -1;
+    }
+
+    // ---- previous row: normalisers, bonus screen (only the pending draft exps are live)
     float scT = 0.f, scD = 0.f;
-    bool prev_bonus = false;
-    if (prev_valid) {
-      const int64_t pit = it - 1;
-      const int pslot = (int)(pit % kRing);
-      const int pk = (int)(pit % a.R);
-      const int64_t punit = cid + (pit / a.R) * G;
+    if (prev) {
+      const int pit = it - 1;
+      const int pslot = pit % kRing;
+      const int pk = k == 0 ? a.R - 1 : k - 1;
+      const int64_t punit = k == 0 ? unit - G : unit;
       if (!mbar_wait(&tl->rbar[pslot], (uint32_t)((pit / kRing) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
       const Msg* rv = tl->recv[pslot];
       const bool has = lane < (int)C;
-      const float pm1 = has ? rv[lane].mT : -INFINITY, ps1 = has ? rv[lane].sT : 0.f;
-      const float pm2 = has ? rv[lane].mD : -INFINITY, ps2 = has ? rv[lane].sD : 0.f;
-      const float MT = warp_max(pm1), MD = warp_max(pm2);
-      const float ST = warp_sum(part_term(pm1, ps1, MT, a.cT));
-      const float SD = warp_sum(part_term(pm2, ps2, MD, a.cT));
-      const bool badT = !(MT > -INFINITY && MT < INFINITY && ST > 0.f && ST < INFINITY);
-      const bool badD = !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
-      scT = (!badT && okT_p) ? ex2((mwT_p - MT) * a.cT) / ST : 0.f;
-      scD = (!badD && okD_p) ? ex2((mwD_p - MD) * a.cT) / SD : 0.f;
+      const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
+                               has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, a.cT);
+      scT = (!nm.badT && okT_p) ? ex2((mwT_p - nm.MT) * a.cT) / nm.ST : 0.f;
+      scD = (!nm.badD && okD_p) ? ex2((mwD_p - nm.MD) * a.cT) / nm.SD : 0.f;
       if (pk == a.K) {
-        prev_bonus = true;
         Cand cd = cand_empty();
-        if (!badT && okT_p) {
+        if (!nm.badT && okT_p) {
           // Tref = M/tau + g_min - margin: a lower bound on the winning score.
-          const float margin = 1e-5f + 2e-7f * fabsf(MT * inv_tau);
-          const float rho = ex2((mwT_p - MT) * a.cT + (-kGumbelMinF + margin) * kLog2e);
+          const float margin = 1e-5f + 2e-7f * fabsf(nm.MT * inv_tau);
+          const float rho = ex2((mwT_p - nm.MT) * a.cT + (-kGumbelMinF + margin) * kLog2e);
+          const float mw_a = mwT_p * inv_tau;
           const Stream st(a.seed, a.round, SD_STREAM_BONUS);
 #pragma unroll
           for (int q = 0; q < EPT / 4; ++q) {
@@ -1400,7 +1477,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
             const bool k1 = keep_bonus(y1, u1) && e0 + 1 < len;
             const bool k2 = keep_bonus(y2, u2) && e0 + 2 < len;
             const bool k3 = keep_bonus(y3, u3) && e0 + 3 < len;
-            const float mw_a = mwT_p * inv_tau;
             if (k0 | k1 | k2 | k3) {
               if (k0) cd = cand_merge(cd, bonus_cand(ev.x, u0, mw_a, v0));
               if (k1) cd = cand_merge(cd, bonus_cand(ev.y, u1, mw_a, v0 + 1));
@@ -1411,78 +1487,58 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
         }
         cd = warp_cand(cd);
         if (lane == 0) tl->wcand[par][warp] = cd;
-        (void)punit;
       }
     }
 
+    // ---- current row: ring -> registers, maxima
+    float mwT = -INFINITY, mwD = -INFINITY;
+    if (cur) {
+      if (!mbar_wait(&tl->full[par], (uint32_t)((it >> 1) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+      const int64_t row = unit * a.R + k;
+      const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes);
+      const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes + a.stage_bytes);
+      const TIn* gT = (const TIn*)a.zT + row * a.ld + s0;
+      const TIn* gD = (const TIn*)a.zD + row * a.ld + s0;
+      mwT = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, tid, ncomp);
+      mwD = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, tid, ncomp);
+      if (x >= s0 && x < s0 + len) {
+        const int le = x - s0;
+        if (((le / EPC) % ncomp) == tid) {
+          tl->zx[par][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
+          tl->zx[par][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
+        }
+      }
+      warp_max2(mwT, mwD);
+    }
+    const float mwTs = mwT == -INFINITY ? 0.f : mwT;
+    const float mwDs = mwD == -INFINITY ? 0.f : mwD;
+
     // ---- fused pass: row r exps + row r-1 TV ----
     float sT = 0.f, sD = 0.f, tv = 0.f;
-    if (cur && prev_valid)
+    if (cur && prev)
       fused_pass<CPT, EPC, true, true>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD, sT,
                                        sD, tv);
     else if (cur)
       fused_pass<CPT, EPC, true, false>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD,
                                         sT, sD, tv);
-    else
+    else if (prev)
       fused_pass<CPT, EPC, false, true>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD,
                                         sT, sD, tv);
-    sT = warp_sum(sT);
-    sD = warp_sum(sD);
-    tv = warp_sum(tv);
+    warp_sum3(sT, sD, tv);
     if (lane == 0) {
       tl->wpart[par][warp] = make_float4(mwT, sT, mwD, sD);
       tl->tvw[par][warp] = tv;
     }
-    bar_sync_n(1, ncomp);  // (A) warp partials visible; this row's stage is free
-    if (cur && tid == 0 && it + 2 < nrows) issue(it + 2);
-    if (warp == 0) {
-      const float tvp = lane < nwarps ? tl->tvw[par][lane] : 0.f;
-      const float tvc = want_tv ? warp_sum(tvp) : 0.f;
-      if (cur) {
-        const float4 wp =
-            lane < nwarps ? tl->wpart[par][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
-        Msg m;
-        m.mT = warp_max(wp.x);
-        m.mD = warp_max(wp.z);
-        m.sT = warp_sum(part_term(wp.x, wp.y, m.mT, a.cT));
-        m.sD = warp_sum(part_term(wp.z, wp.w, m.mD, a.cT));
-        m.tvprev = tvc;
-        m.aux = 0;
-        m.zxT = owner ? tl->zx[par][0] : 0.f;
-        m.zxD = owner ? tl->zx[par][1] : 0.f;
-        const int slot = (int)(it % kRing);
-        if (leader && it >= 2 && !mbar_wait(&tl->bdone[(it - 2) % kRing], (uint32_t)(((it - 2) / kRing) & 1)))
-          raise_err(a.dev_err, SD_DEV_TIMEOUT);
-        if (lane == 0) mbar_arrive_expect_tx(&tl->rbar[slot], C * (uint32_t)sizeof(Msg));
-        if (lane < (int)C) {
-          const uint32_t ra = peer_addr(&tl->recv[slot][rank], (uint32_t)lane);
-          const uint32_t rb = peer_addr(&tl->rbar[slot], (uint32_t)lane);
-          st_async_v4(ra, m.mT, m.sT, m.mD, m.sD, rb);
-          st_async_v4(ra + 16, m.zxT, m.zxD, m.tvprev, 0.f, rb);
-        }
-      } else if (want_tv && prev_valid) {  // final iteration: the last row's TV goes to the leader
-        if (leader && lane == 0) mbar_arrive_expect_tx(&tl->fbar, C * 4u);
-        if (lane == 0)
-          st_async_b32(peer_addr(&tl->frecv[rank], 0), __float_as_uint(tvc), peer_addr(&tl->fbar, 0));
-      }
-      if (prev_bonus) {  // row r-1's bonus candidate goes to the leader
-        const int pslot = (int)((it - 1) % kRing);
-        Cand c2 = lane < nwarps ? tl->wcand[par][lane] : cand_empty();
-        c2 = warp_cand(c2);
-        if (leader && lane == 0) mbar_arrive_expect_tx(&tl->cbar[pslot], C * (uint32_t)sizeof(Cand));
-        if (lane == 0) {
-          const uint32_t ra = peer_addr(&tl->crecv[pslot][rank], 0);
-          const uint32_t rb = peer_addr(&tl->cbar[pslot], 0);
-          st_async_v4(ra, c2.s, c2.lo, c2.hi, c2.ohi, rb);
-          st_async_v4(ra + 16, __int_as_float(c2.idx), 0.f, 0.f, 0.f, rb);
-        }
-      }
-    }
+    // (A) post this iteration's partials to the communication warp and move on
+    asm volatile("bar.arrive 1, %0;" ::"r"(ncomp + 32) : "memory");
     mwT_p = mwTs;
     mwD_p = mwDs;
     okT_p = mwT > -INFINITY;
     okD_p = mwD > -INFINITY;
-    prev_valid = cur;
+    if (cur && ++k == a.R) {
+      k = 0;
+      unit += G;
+    }
   }
   cluster_sync();
 }
@@ -1607,7 +1663,7 @@ static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, Launc
   for (int C = 1; C <= kMaxCluster; ++C) {
     const int slice = (int)(((int64_t)(V + C - 1) / C + 7) / 8 * 8);
     const int ncomp = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
-    const int threads = ncomp + 32;
+    const int threads = ncomp + 64;  // + communication and bookkeeping warps
     if (threads > kMaxThreads || ncomp / 32 > kMaxWarps) continue;
     const uint32_t sb = (uint32_t)(((int64_t)slice * esize + 127) / 128 * 128);
     const size_t smem = (size_t)2 * 2 * sb + (size_t)ncomp * kEPT * 4 + sizeof(SmcTail) + 128;

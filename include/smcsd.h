@@ -69,6 +69,9 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_DEV_PAGE_OOB 8u       /* page id outside [0, num_pages) and != -1   */
 #define SD_DEV_ANCESTOR_OOB 16u  /* ancestor index outside [0, N)              */
 #define SD_DEV_TIMEOUT 32u       /* an internal bounded wait gave up           */
+/* With SD_DEV_TIMEOUT, smcsd_score also sets one of bits 8..15 naming the
+ * wait that gave up (diagnostic only; outputs of that call are invalid). */
+#define SD_DEV_WAIT_SITE_MASK 0xFF00u
 
 /* Philox stream tags. */
 #define SD_STREAM_BONUS 1u

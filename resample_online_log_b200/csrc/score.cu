@@ -53,7 +53,7 @@ struct ScoreArgs {
   int64_t units;
   int slice;             // entries per group slice (a multiple of 8)
   int groups;            // independent warp groups per CTA (1..3)
-  int stages;
+  int stages;            // ring stages
   uint32_t stage_bytes;  // bytes reserved for one tensor's slice in a stage
   int use_tma;
   float inv_tau, cT;     // 1/tau and log2(e)/tau, fp32
@@ -1029,38 +1029,76 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
 }
 
 // ====================================================================== SMC-SD kernel
-// Software-pipelined variant for SMC-SD rounds (every row has a target and a
-// draft half, the last row of each particle draws the bonus token).
+// Pipelined kernel for SMC-SD rounds: every row has a target and a draft half;
+// the last row of each particle also draws the bonus token.  A cluster of C
+// CTAs walks its particles' rows in order; CTA r owns vocabulary slice r.
 //
-// Iteration r of a CTA:
-//   1. move row r's slices from the ring to registers, per-thread and warp max;
-//   2. wait for row r-1's messages (sent one iteration ago, so their latency is
-//      hidden behind step 1), rebuild row r-1's normalisers, screen row r-1's
-//      bonus candidates if it ends a particle;
-//   3. one fused loop over this thread's entries: row r's exp2 (MUFU) and sums,
-//      row r-1's TV from its target exps (shared-memory buffer) and draft exps
-//      (registers) -- each slot is read and then overwritten in place;
-//   4. one CTA barrier; warp 0 combines the warp partials and pushes row r's
-//      message (carrying row r-1's TV partial) to every CTA of the cluster, and
-//      row r-1's bonus candidate to the leader.
-// Row r's exps thus stay on chip until its TV is taken one iteration later;
-// the bookkeeping warp of the leader turns the messages into log-weights, TV
-// and bonus tokens (deciding near-ties exactly in fp64).
+// Iteration `it` of the compute warps has two phases:
+//   A(it)    row it: move its slices from the ring to registers, warp maxima,
+//            exps (one MUFU exp2 per entry) and sums; the exps of both halves
+//            go to tensor memory (TMEM), two row buffers per warp.  The
+//            compute warps then meet at one barrier and post their (max, sum)
+//            partials.
+//   B(it-1)  row it-1: wait for its messages from the cluster (sent during
+//            phase A, so the exchange is hidden behind it), rebuild the row
+//            normalisers, read the row's exps back from TMEM and take the TV
+//            partial sum |p - q|; on a particle's last row also screen the
+//            bonus-token candidates.
+// A communication warp turns the warp partials into one 32-byte message per
+// row for every CTA of the cluster (st.async into distributed shared memory,
+// completing on the receiver's mbarrier -- no cluster barrier on the row
+// path), sends each row's TV partial and bonus candidate to the leader, and
+// refills the ring with bulk async copies (no multicast) once phase A has
+// released a stage.  The leader's bookkeeping warp turns the messages into
+// fp64 lse, log-probs, log-weights, TV and bonus tokens (near-ties settled
+// exactly in fp64).  Every element is read from HBM once and exponentiated once.
 
-constexpr int kRing = 4;  // message slots: the bookkeeping warp may lag two rows
+constexpr int kRing = 8;     // message slots per CTA
+constexpr int kLead = 2;     // rows a CTA's messages can run ahead of the leader's
+constexpr int kMaxStages = 4;
+constexpr uint32_t kTmemCols = 512;  // all of the SM's tensor memory (one CTA per SM)
+constexpr size_t kMinSmem = 120 * 1024;  // > half an SM's shared memory: one CTA per SM
+
+struct alignas(16) BMsg {  // one slice's phase-B results for the leader
+  float tv, s, lo, hi;
+  float ohi;
+  int idx;
+  float pad0, pad1;
+};
 
 struct alignas(128) SmcTail {
-  uint64_t full[2];
-  uint64_t rbar[kRing], cbar[kRing], bdone[kRing];
-  uint64_t fbar, pad;
+  uint64_t full[kMaxStages];    // ring stages (target and draft slices of one row)
+  uint64_t afull[2], bfull[2];  // compute warps -> communication warp, by row parity
+  uint64_t rbar[kRing], bbar[kRing], adone[kRing];
+  int abort_flag;
+  uint32_t tmem_base;
   Msg recv[kRing][kMaxCluster];
-  Cand crecv[kRing][kMaxCluster];
-  float frecv[kMaxCluster];
-  float4 wpart[2][kMaxWarps];  // warp scratch, by iteration parity: warps may run one
-  float tvw[2][kMaxWarps];     // iteration ahead of warp 0, which reads the previous one
+  BMsg brecv[kRing][kMaxCluster];
+  float4 wpart[2][kMaxWarps];
+  float wtv[2][kMaxWarps];
   Cand wcand[2][kMaxWarps];
   float zx[2][2];
 };
+
+// Wait sites, reported in bits 8..15 of the error word with SD_DEV_TIMEOUT.
+enum WaitSite : uint32_t {
+  kWsFull = 1u << 8, kWsRow = 1u << 10, kWsAfull = 1u << 11, kWsBfull = 1u << 12,
+  kWsAdone = 1u << 13, kWsBook = 1u << 14, kWsBmsg = 1u << 15
+};
+
+// Bounded wait; after one expiry every later wait of the CTA returns at once
+// (the outputs are then garbage, SD_DEV_TIMEOUT is set, nothing hangs).
+__device__ __forceinline__ void swait(uint64_t* bar, uint32_t parity, SmcTail* tl, uint32_t* err,
+                                      uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return;
+  volatile int* ab = &tl->abort_flag;
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (*ab) return;
+    if (mbar_try_wait(bar, parity)) return;
+  }
+  *ab = 1;
+  raise_err(err, SD_DEV_TIMEOUT | site);
+}
 
 // Paired warp reductions (two independent values per shuffle round).
 __device__ __forceinline__ void warp_max2(float& a, float& b) {
@@ -1072,6 +1110,15 @@ __device__ __forceinline__ void warp_max2(float& a, float& b) {
     b = fmaxf(b, y);
   }
 }
+__device__ __forceinline__ void warp_max2_nan(float& a, float& b) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float x = __shfl_xor_sync(0xffffffffu, a, o);
+    const float y = __shfl_xor_sync(0xffffffffu, b, o);
+    a = fmax_nan(a, x);
+    b = fmax_nan(b, y);
+  }
+}
 __device__ __forceinline__ void warp_sum2(float& a, float& b) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -1081,23 +1128,31 @@ __device__ __forceinline__ void warp_sum2(float& a, float& b) {
     b += y;
   }
 }
-__device__ __forceinline__ void warp_sum3(float& a, float& b, float& c) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float x = __shfl_xor_sync(0xffffffffu, a, o);
-    const float y = __shfl_xor_sync(0xffffffffu, b, o);
-    const float z = __shfl_xor_sync(0xffffffffu, c, o);
-    a += x;
-    b += y;
-    c += z;
-  }
-}
 // fp64 lse of a row from per-slice partials (one per lane, `has` marks valid
 // lanes); the slice factors use MUFU exp2, the sum and the log are fp64.
 __device__ __noinline__ double row_lse_fast(float m, float s, float M, bool has, double tau64,
                                             float cT) {
   const double t = (has && m > -INFINITY) ? (double)s * (double)ex2((m - M) * cT) : 0.0;
   return (double)M / tau64 + log(warp_sum_d(t));
+}
+
+// Row normalisers from per-slice (max, sum) partials held one per lane.  A
+// NaN partial max drops out of the max but makes the sum NaN.
+struct Norm {
+  float MT, ST, MD, SD;
+  bool badT, badD;
+};
+__device__ __forceinline__ Norm row_norm(float pm1, float ps1, float pm2, float ps2, float cT) {
+  Norm n;
+  n.MT = pm1;
+  n.MD = pm2;
+  warp_max2(n.MT, n.MD);
+  n.ST = part_term(pm1, ps1, n.MT, cT);
+  n.SD = part_term(pm2, ps2, n.MD, cT);
+  warp_sum2(n.ST, n.SD);
+  n.badT = !(n.MT > -INFINITY && n.MT < INFINITY && n.ST > 0.f && n.ST < INFINITY);
+  n.badD = !(n.MD > -INFINITY && n.MD < INFINITY && n.SD > 0.f && n.SD < INFINITY);
+  return n;
 }
 
 // Exact fp64 bonus draw over a whole target row (a near-tie the fp32 screen
@@ -1127,182 +1182,268 @@ __device__ __noinline__ int exact_bonus_row(const TIn* row, int V, double tau64,
   return bi == 0x7FFFFFFF ? -1 : bi;
 }
 
+// Candidate from one kept entry: a = z / tau in fp32, Gumbel in fp32, with
+// bounds that contain the exact fp64 score.
+__device__ __noinline__ Cand bonus_cand_z(float z, float u, float inv_tau, int v) {
+  const float g32 = gumbel_f32(u);
+  const float a32 = z * inv_tau;
+  Cand cd;
+  cd.s = a32 + g32;
+  const float d = 4e-6f + 4.8e-7f * (fabsf(a32) + 2.f * fabsf(g32));
+  cd.lo = cd.s - d;
+  cd.hi = cd.s + d;
+  cd.ohi = -INFINITY;
+  cd.idx = v;
+  cd.pad0 = cd.pad1 = cd.pad2 = 0;
+  return cd;
+}
+
+// 16-byte chunks of a row slice: 8 bf16 or 4 fp32 entries.
+template <typename TIn>
+struct Chunk;
+template <>
+struct Chunk<uint16_t> {
+  static constexpr int EPC = 8;
+  using Acc = uint32_t;  // two bf16 maxima
+  static constexpr uint32_t kAcc0 = 0xFF80FF80u;
+  static __device__ __forceinline__ void max_acc(Acc& m, const uint4& v) {
+    m = bmax2_nan(m, bmax2_nan(bmax2_nan(v.x, v.y), bmax2_nan(v.z, v.w)));
+  }
+  static __device__ __forceinline__ float acc_f32(Acc m) {
+    return fmax_nan(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+  }
+  static __device__ __forceinline__ float elem(const uint4& v, int j) {  // j: compile-time
+    const uint32_t w = (j >> 1) == 0 ? v.x : ((j >> 1) == 1 ? v.y : ((j >> 1) == 2 ? v.z : v.w));
+    return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
+  }
+  static __device__ __noinline__ uint4 gather(const uint16_t* st, const uint16_t* g, int e0, int len,
+                                              int tma_len) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t h[2];
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const int e = e0 + 2 * j + b;
+        h[b] = e < tma_len ? (uint32_t)st[e] : (e < len ? (uint32_t)g[e] : 0xFF80u);
+      }
+      w[j] = h[0] | (h[1] << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+template <>
+struct Chunk<float> {
+  static constexpr int EPC = 4;
+  using Acc = float;
+  static constexpr float kAcc0 = -INFINITY;
+  static __device__ __forceinline__ void max_acc(Acc& m, const uint4& v) {
+    m = fmax_nan(m, fmax_nan(fmax_nan(__uint_as_float(v.x), __uint_as_float(v.y)),
+                             fmax_nan(__uint_as_float(v.z), __uint_as_float(v.w))));
+  }
+  static __device__ __forceinline__ float acc_f32(Acc m) { return m; }
+  static __device__ __forceinline__ float elem(const uint4& v, int j) {  // j: compile-time
+    return __uint_as_float(j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w)));
+  }
+  static __device__ __noinline__ uint4 gather(const float* st, const float* g, int e0, int len,
+                                              int tma_len) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + j;
+      w[j] = e < tma_len ? __float_as_uint(st[e])
+                         : (e < len ? __float_as_uint(g[e]) : 0xFF800000u);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+// Chunk starting at slice entry e0: from the ring stage where the bulk copy
+// covered it, else from HBM; entries past the slice read as -inf.
+template <typename TIn>
+__device__ __forceinline__ uint4 load_chunk(const TIn* st, const TIn* g, int e0, int len,
+                                            int tma_len) {
+  if (e0 + Chunk<TIn>::EPC <= tma_len) return *reinterpret_cast<const uint4*>(st + e0);
+  return Chunk<TIn>::gather(st, g, e0, len, tma_len);
+}
+
+// Bonus-token screen over this thread's target entries of a particle's last
+// row, from the exps held in TMEM (relative to the warp max): entries whose
+// y = e * rho = e^{a - Tref} proves they cannot win are dropped before any
+// log, groups of four far below Tref before the Philox call; the few kept
+// entries re-read their logit from HBM and become candidates with fp32
+// bounds.  Its loop stays rolled: one row in K+1 needs it.
+template <typename TIn>
+__device__ __forceinline__ Cand bonus_screen(uint32_t tcolT, const TIn* g, int s0, int len, int tid,
+                                             int ncomp, float rho, float inv_tau, const Stream bst,
+                                             uint32_t rowid) {
+  constexpr int EPC = Chunk<TIn>::EPC;
+  Cand cd = cand_empty();
+#pragma unroll 1
+  for (int i8 = 0; i8 < kEPT; i8 += 8) {
+    float e[8];
+    __syncwarp();  // converge after the divergent screening of the previous block
+    tmem_ld8(tcolT + (uint32_t)i8, e);
+    tmem_wait_ld();
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int i = i8 + 4 * q;  // this thread's entry index: chunk i / EPC, offset i % EPC
+      const int eg = (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
+      float y[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) y[j] = e[4 * q + j] * rho;
+      if (eg >= len || fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3])) < kYSkip) continue;
+      const int v0 = s0 + eg;
+      const U4 w = bst.at((uint32_t)(v0 >> 2), rowid);
+      const float u[4] = {uniform_f32(w.x), uniform_f32(w.y), uniform_f32(w.z), uniform_f32(w.w)};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (!keep_bonus(y[j], u[j]) || eg + j >= len) continue;
+        const float z = Elem<TIn>::get(g, eg + j);
+        if (z > -INFINITY) cd = cand_merge(cd, bonus_cand_z(z, u[j], inv_tau, v0 + j));
+      }
+    }
+  }
+  return cd;
+}
+
 template <typename TIn>
 __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32_t cid, uint32_t G,
                              int nrows, bool want_tv) {
   const int lane = threadIdx.x & 31;
+  const Stream bst(a.seed, a.round, SD_STREAM_BONUS);
+  const bool lane_tokens = a.K <= 32;
   double logw_acc = 0.0;
   bool unit_bad = false;
-  bool prev_bad = false;
-  int cuse[kRing] = {0, 0, 0, 0};
-  const Stream bst(a.seed, a.round, SD_STREAM_BONUS);
+  bool prev_bad = false, prev_badT = false;
   int k = 0;
   int64_t unit = cid;
-  int64_t prev_row = -1;
-  for (int it = 0; it < nrows; ++it, prev_row = unit * a.R + k, (++k == a.R ? (k = 0, unit += G) : 0)) {
-    const int slot = it % kRing;
-    const int64_t rowT = unit * a.R + k;
-    if (!mbar_wait(&tl->rbar[slot], (uint32_t)((it / kRing) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
-    const Msg* e = tl->recv[slot];
-    const bool has = lane < (int)C;
-    const float pm1 = has ? e[lane].mT : -INFINITY, ps1 = has ? e[lane].sT : 0.f;
-    const float pm2 = has ? e[lane].mD : -INFINITY, ps2 = has ? e[lane].sD : 0.f;
-    float tvsum = has ? e[lane].tvprev : 0.f;
-    float MT = pm1, MD = pm2;
-    warp_max2(MT, MD);
-    float ST = part_term(pm1, ps1, MT, a.cT), SD = part_term(pm2, ps2, MD, a.cT);
-    warp_sum3(ST, SD, tvsum);
-    const bool badT = !(MT > -INFINITY && MT < INFINITY && ST > 0.f && ST < INFINITY);
-    const bool badD = !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
-    const bool bad = badT || badD;
-    const double lse64T = row_lse_fast(pm1, ps1, MT, has, a.tau64, a.cT);
-    const double lse64D = row_lse_fast(pm2, ps2, MD, has, a.tau64, a.cT);
-    int x = -1;
-    float zxT = 0.f, zxD = 0.f;
-    if (k < a.K) {
-      x = a.draft[unit * a.K + k];
-      if (x >= 0 && x < a.V) {
-        const Msg& o = e[x / a.slice];
-        zxT = o.zxT;
-        zxD = o.zxD;
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&tl->bdone[slot]);  // message slot no longer needed
-    if (lane == 0) {
+  // draft tokens of a particle, one per lane; prefetched one particle ahead
+  auto fetch_tokens = [&](int64_t u) -> int {
+    return (lane_tokens && lane < a.K && u < a.units) ? a.draft[u * a.K + lane] : -1;
+  };
+  auto fetch_prev = [&](int64_t u) -> double {
+    return (a.logw_prev && u < a.units) ? a.logw_prev[u] : 0.0;
+  };
+  int xs = -1, xs_next = fetch_tokens(unit);
+  double lwp = 0.0, lwp_next = fetch_prev(unit);
+  for (int it = 0; it <= nrows; ++it) {
+    bool bad_cur = false, badT_cur = false;
+    if (it < nrows) {
       if (k == 0) {
+        xs = xs_next;
+        lwp = lwp_next;
+        xs_next = fetch_tokens(unit + G);
+        lwp_next = fetch_prev(unit + G);
         logw_acc = 0.0;
         unit_bad = false;
       }
-      if (it > 0 && want_tv) a.tv_out[prev_row] = prev_bad ? NAN : 0.5f * tvsum;
-      if (bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
-      if (a.lse_out) {
-        a.lse_out[rowT * 2 + 0] = badT ? NAN : lse64T;
-        a.lse_out[rowT * 2 + 1] = badD ? NAN : lse64D;
-      }
+      const int slot = it % kRing;
+      const int64_t rowT = unit * a.R + k;
+      swait(&tl->rbar[slot], (uint32_t)((it / kRing) & 1), tl, a.dev_err, kWsBook);
+      const Msg* e = tl->recv[slot];
+      const bool has = lane < (int)C;
+      const Norm nm = row_norm(has ? e[lane].mT : -INFINITY, has ? e[lane].sT : 0.f,
+                               has ? e[lane].mD : -INFINITY, has ? e[lane].sD : 0.f, a.cT);
+      const double lse64T = row_lse_fast(has ? e[lane].mT : -INFINITY, has ? e[lane].sT : 0.f,
+                                         nm.MT, has, a.tau64, a.cT);
+      const double lse64D = row_lse_fast(has ? e[lane].mD : -INFINITY, has ? e[lane].sD : 0.f,
+                                         nm.MD, has, a.tau64, a.cT);
+      bad_cur = nm.badT || nm.badD;
+      badT_cur = nm.badT;
+      int x = -1;
+      float zxT = 0.f, zxD = 0.f;
       if (k < a.K) {
-        const bool x_ok = x >= 0 && x < a.V;
-        double lp = NAN, lq = NAN;
-        if (!x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
-        if (x_ok && !bad) {
-          lp = (double)zxT / a.tau64 - lse64T;
-          lq = (double)zxD / a.tau64 - lse64D;
-        } else {
-          unit_bad = true;
+        x = lane_tokens ? __shfl_sync(0xffffffffu, xs, k) : a.draft[unit * a.K + k];
+        if (x >= 0 && x < a.V) {
+          const Msg& o = e[x / a.slice];
+          zxT = o.zxT;
+          zxD = o.zxD;
         }
-        logw_acc += lp - lq;
-        if (a.lp_out) {
-          a.lp_out[(unit * a.K + k) * 2 + 0] = lp;
-          a.lp_out[(unit * a.K + k) * 2 + 1] = lq;
-        }
-      } else {
-        const double prev = a.logw_prev ? a.logw_prev[unit] : 0.0;
-        a.logw_out[unit] = unit_bad ? NAN : prev + logw_acc;
-        if (a.tokens_out)
-          for (int jj = 0; jj < a.K; ++jj) a.tokens_out[unit * a.R + jj] = a.draft[unit * a.K + jj];
       }
-    }
-    prev_bad = bad;
-    if (k == a.K) {  // bonus token: merge the slices' candidates
-      const uint32_t ph = (uint32_t)(cuse[slot] & 1);
-      ++cuse[slot];
-      if (!mbar_wait(&tl->cbar[slot], ph)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
-      Cand c = has ? tl->crecv[slot][lane] : cand_empty();
-      c = warp_cand(c);
-      int winner;
-      if (badT || c.idx == 0x7FFFFFFF) winner = -1;
-      else if (c.ohi < c.lo) winner = c.idx;
-      else
-        winner = exact_bonus_row<TIn>((const TIn*)a.zT + rowT * a.ld, a.V, a.tau64, a.inv_tau, c.lo,
-                                      bst, (uint32_t)unit);
       __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->adone[slot]);  // this row's message slot is read
       if (lane == 0) {
-        a.bonus_out[unit] = winner;
-        if (a.tokens_out) a.tokens_out[unit * a.R + a.K] = winner;
-      }
-    }
-  }
-  if (want_tv && nrows > 0) {  // the last row's TV arrives on its own
-    if (!mbar_wait(&tl->fbar, 0)) raise_err(a.dev_err, SD_DEV_TIMEOUT);
-    float v = lane < (int)C ? tl->frecv[lane] : 0.f;
-    v = warp_sum(v);
-    if (lane == 0) a.tv_out[prev_row] = prev_bad ? NAN : 0.5f * v;
-  }
-}
-
-// Fused per-thread pass: row r's exps (CUR) and row r-1's TV (PREV).
-template <int CPT, int EPC, bool CUR, bool PREV>
-__device__ __forceinline__ void fused_pass(float* xt, float* xd, float* dp, float4* tb, int tid,
-                                           int nthr, float mwT, float mwD, float cT, float scT,
-                                           float scD, float& sT, float& sD, float& tv) {
-  constexpr int EPT = CPT * EPC;
-  float2 aT = make_float2(0.f, 0.f), aD = make_float2(0.f, 0.f);
-  float t0 = 0.f, t1 = 0.f;
-  const float2 mT2 = make_float2(-mwT, -mwT), mD2 = make_float2(-mwD, -mwD);
-  const float2 c2 = make_float2(cT, cT);
-#pragma unroll
-  for (int q = 0; q < EPT / 4; ++q) {
-    float4& slot = tb[q * nthr + tid];
-    float4 old = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (PREV) old = slot;
-    float4 nw;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = q * 4 + h * 2;
-      if (PREV) {  // separately rounded products: identical rows give exactly 0
-        const float o0 = h == 0 ? old.x : old.z, o1 = h == 0 ? old.y : old.w;
-        t0 += fabsf(__fmul_rn(o0, scT) - __fmul_rn(dp[i], scD));
-        t1 += fabsf(__fmul_rn(o1, scT) - __fmul_rn(dp[i + 1], scD));
-      }
-      if (CUR) {
-        const float2 at = __fmul2_rn(__fadd2_rn(make_float2(xt[i], xt[i + 1]), mT2), c2);
-        const float2 ad = __fmul2_rn(__fadd2_rn(make_float2(xd[i], xd[i + 1]), mD2), c2);
-        const float2 et = make_float2(ex2(at.x), ex2(at.y));
-        const float2 ed = make_float2(ex2(ad.x), ex2(ad.y));
-        aT = __fadd2_rn(aT, et);
-        aD = __fadd2_rn(aD, ed);
-        if (h == 0) {
-          nw.x = et.x;
-          nw.y = et.y;
-        } else {
-          nw.z = et.x;
-          nw.w = et.y;
+        if (bad_cur) raise_err(a.dev_err, SD_DEV_NONFINITE);
+        if (a.lse_out) {
+          a.lse_out[rowT * 2 + 0] = nm.badT ? NAN : lse64T;
+          a.lse_out[rowT * 2 + 1] = nm.badD ? NAN : lse64D;
         }
-        dp[i] = ed.x;
-        dp[i + 1] = ed.y;
+        if (k < a.K) {
+          const bool x_ok = x >= 0 && x < a.V;
+          double lp = NAN, lq = NAN;
+          if (!x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
+          if (x_ok && !bad_cur) {
+            lp = (double)zxT / a.tau64 - lse64T;
+            lq = (double)zxD / a.tau64 - lse64D;
+          } else {
+            unit_bad = true;
+          }
+          logw_acc += lp - lq;
+          if (a.lp_out) {
+            a.lp_out[(unit * a.K + k) * 2 + 0] = lp;
+            a.lp_out[(unit * a.K + k) * 2 + 1] = lq;
+          }
+        } else {
+          a.logw_out[unit] = unit_bad ? NAN : lwp + logw_acc;
+        }
+      }
+      if (k == a.K && a.tokens_out) {
+        if (lane_tokens) {
+          if (lane < a.K) a.tokens_out[unit * a.R + lane] = xs;
+        } else {
+          for (int j = lane; j < a.K; j += 32) a.tokens_out[unit * a.R + j] = a.draft[unit * a.K + j];
+        }
       }
     }
-    if (CUR) slot = nw;
+    if (it >= 1) {  // row it-1: TV partials and the bonus candidates
+      const int p = it - 1;
+      const int pslot = p % kRing;
+      const int pk = k == 0 ? a.R - 1 : k - 1;
+      const int64_t punit = k == 0 ? unit - G : unit;
+      swait(&tl->bbar[pslot], (uint32_t)((p / kRing) & 1), tl, a.dev_err, kWsBmsg);
+      const BMsg* bm = tl->brecv[pslot];
+      const bool has = lane < (int)C;
+      float tv = has ? bm[lane].tv : 0.f;
+      tv = warp_sum(tv);
+      if (want_tv && lane == 0) a.tv_out[punit * a.R + pk] = prev_bad ? NAN : 0.5f * tv;
+      if (pk == a.K) {
+        Cand c = cand_empty();
+        if (has) {
+          c.s = bm[lane].s;
+          c.lo = bm[lane].lo;
+          c.hi = bm[lane].hi;
+          c.ohi = bm[lane].ohi;
+          c.idx = bm[lane].idx;
+        }
+        c = warp_cand(c);
+        int winner;
+        if (prev_badT || c.idx == 0x7FFFFFFF) winner = -1;
+        else if (c.ohi < c.lo) winner = c.idx;
+        else
+          winner = exact_bonus_row<TIn>((const TIn*)a.zT + (punit * a.R + pk) * a.ld, a.V, a.tau64,
+                                        a.inv_tau, c.lo, bst, (uint32_t)punit);
+        if (lane == 0) {
+          a.bonus_out[punit] = winner;
+          if (a.tokens_out) a.tokens_out[punit * a.R + a.K] = winner;
+        }
+      }
+    }
+    prev_bad = bad_cur;
+    prev_badT = badT_cur;
+    if (it < nrows && ++k == a.R) {
+      k = 0;
+      unit += G;
+    }
   }
-  sT = aT.x + aT.y;
-  sD = aD.x + aD.y;
-  tv = t0 + t1;
-  (void)EPC;
 }
 
-// Row normalisers from per-slice (max, sum) partials held one per lane.
-struct Norm {
-  float MT, ST, MD, SD;
-  bool badT, badD;
-};
-__device__ __forceinline__ Norm row_norm(float pm1, float ps1, float pm2, float ps2, float cT) {
-  Norm n;
-  n.MT = pm1;
-  n.MD = pm2;
-  warp_max2(n.MT, n.MD);
-  n.ST = part_term(pm1, ps1, n.MT, cT);
-  n.SD = part_term(pm2, ps2, n.MD, cT);
-  warp_sum2(n.ST, n.SD);
-  n.badT = !(n.MT > -INFINITY && n.MT < INFINITY && n.ST > 0.f && n.ST < INFINITY);
-  n.badD = !(n.MD > -INFINITY && n.MD < INFINITY && n.SD > 0.f && n.SD < INFINITY);
-  return n;
-}
-
-template <typename TIn, int CPT>
+template <typename TIn>
 __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) {
-  constexpr int EPC = 16 / (int)sizeof(TIn);
-  constexpr int EPT = CPT * EPC;
-  static_assert(EPT == kEPT, "entries per thread");
+  using CK = Chunk<TIn>;
+  constexpr int EPC = CK::EPC;
+  constexpr int CPT = kEPT / EPC;          // chunks per thread
+  constexpr bool HOLD = sizeof(TIn) == 2;  // bf16: raw chunks stay in registers for pass 2
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1310,9 +1451,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
   const int ncomp = blockDim.x - 64, nwarps = ncomp >> 5;
   const uint32_t rank = cluster_rank(), C = cluster_size();
   const uint32_t cid = cluster_id(), G = num_clusters();
-  float4* tbuf = reinterpret_cast<float4*>(smem + (size_t)2 * 2 * a.stage_bytes);
-  SmcTail* tl = reinterpret_cast<SmcTail*>(smem + (size_t)2 * 2 * a.stage_bytes +
-                                           (size_t)ncomp * EPT * sizeof(float));
+  const int nS = a.stages;
+  const size_t sb = a.stage_bytes;  // one tensor's slice; a stage holds both
+  SmcTail* tl = reinterpret_cast<SmcTail*>(smem + (size_t)nS * 2 * sb);
 
   const int s0 = (int)rank * a.slice;
   const int len = max(0, min(a.slice, a.V - s0));
@@ -1324,16 +1465,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
   const bool want_tv = a.tv_out != nullptr;
 
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) mbar_init(&tl->full[s], 1);
+    for (int st = 0; st < nS; ++st) mbar_init(&tl->full[st], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tl->afull[b], 1);
+      mbar_init(&tl->bfull[b], (uint32_t)nwarps);
+    }
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&tl->rbar[i], 1);
-      mbar_init(&tl->cbar[i], 1);
-      mbar_init(&tl->bdone[i], 1);
+      mbar_init(&tl->bbar[i], 1);
+      mbar_init(&tl->adone[i], 1);
     }
-    mbar_init(&tl->fbar, 1);
+    tl->abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == nwarps) {  // the communication warp owns the CTA's tensor memory
+    tmem_alloc(&tl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tmem_fence_before();
   __syncthreads();
+  tmem_fence_after();
   cluster_sync();
 
   if (warp == nwarps + 1) {  // ---------------- bookkeeping (leader only)
@@ -1342,92 +1493,100 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
     return;
   }
 
-  const uint64_t pol = policy_evict_first();
-  // stage (row & 1) <- row `it` of this cluster: unit cid + (it / R) * G, position it % R
-  auto issue = [&](int it) {
-    const int s = it & 1;
-    const int64_t row = ((int64_t)cid + (int64_t)(it / a.R) * G) * a.R + (it % a.R);
-    unsigned char* stg = smem + (size_t)s * 2 * a.stage_bytes;
-    mbar_arrive_expect_tx(&tl->full[s], tma_bytes * 2u);
-    if (tma_bytes) {
-      bulk_load(stg, (const TIn*)a.zT + row * a.ld + s0, tma_bytes, &tl->full[s], pol);
-      bulk_load(stg + a.stage_bytes, (const TIn*)a.zD + row * a.ld + s0, tma_bytes, &tl->full[s], pol);
-    }
-  };
-
   if (warp == nwarps) {  // ---------------- communication warp
+    const uint64_t pol = policy_evict_first();
+    // stage st <- row `it` of this cluster: unit cid + (it / R) * G, position it % R
+    auto issue = [&](int it, int st) {
+      const int64_t row = ((int64_t)cid + (int64_t)(it / a.R) * G) * a.R + (it % a.R);
+      unsigned char* stg = smem + (size_t)st * 2 * sb;
+      mbar_arrive_expect_tx(&tl->full[st], 2u * tma_bytes);
+      if (tma_bytes) {
+        bulk_load(stg, (const TIn*)a.zT + row * a.ld + s0, tma_bytes, &tl->full[st], pol);
+        bulk_load(stg + sb, (const TIn*)a.zD + row * a.ld + s0, tma_bytes, &tl->full[st], pol);
+      }
+    };
     if (lane == 0)
-      for (int it = 0; it < nrows && it < 2; ++it) issue(it);
-    int k = 0;
+      for (int i = 0; i < nS && i < nrows; ++i) issue(i, i);
+    int k = 0, stage = 0;  // position and ring stage of row it
     for (int it = 0; it <= nrows; ++it) {
-      const bool cur = it < nrows;
-      const int par = it & 1;
-      bar_sync_n(1, ncomp + 32);  // compute warps have posted their partials of iteration `it`
-      if (cur && lane == 0 && it + 2 < nrows) issue(it + 2);  // stage `par` is free again
-      float tvp = lane < nwarps ? tl->tvw[par][lane] : 0.f;
-      if (cur) {
+      if (it < nrows) {  // row it: phase A done in this CTA; its stage is free
+        swait(&tl->afull[it & 1], (uint32_t)((it >> 1) & 1), tl, a.dev_err, kWsAfull);
+        if (lane == 0 && it + nS < nrows) issue(it + nS, stage);
         const float4 wp =
-            lane < nwarps ? tl->wpart[par][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+            lane < nwarps ? tl->wpart[it & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
         float mT = wp.x, mD = wp.z;
-        warp_max2(mT, mD);
-        float sT = part_term(wp.x, wp.y, mT, a.cT), sD = part_term(wp.z, wp.w, mD, a.cT);
-        warp_sum3(sT, sD, tvp);
-        const bool owner_known = k < a.K;
+        warp_max2_nan(mT, mD);  // a warp's NaN max (NaN in its entries) must reach the sum
+        float sumT = part_term(wp.x, wp.y, mT, a.cT), sumD = part_term(wp.z, wp.w, mD, a.cT);
+        warp_sum2(sumT, sumD);
         float zxT = 0.f, zxD = 0.f;
-        if (owner_known) {
-          zxT = tl->zx[par][0];
-          zxD = tl->zx[par][1];
+        if (k < a.K) {
+          zxT = tl->zx[it & 1][0];
+          zxD = tl->zx[it & 1][1];
         }
         const int slot = it % kRing;
-        if (leader && it >= 2 &&
-            !mbar_wait(&tl->bdone[(it - 2) % kRing], (uint32_t)(((it - 2) / kRing) & 1)))
-          raise_err(a.dev_err, SD_DEV_TIMEOUT);
+        // Once this message is out, the other CTAs can send rows up to it + kLead;
+        // their slots must already have been read by the bookkeeping warp.
+        if (leader && it + kLead >= kRing) {
+          const int r = it + kLead - kRing;
+          swait(&tl->adone[r % kRing], (uint32_t)((r / kRing) & 1), tl, a.dev_err, kWsAdone);
+        }
         if (lane == 0) mbar_arrive_expect_tx(&tl->rbar[slot], C * (uint32_t)sizeof(Msg));
         if (lane < (int)C) {
           const uint32_t ra = peer_addr(&tl->recv[slot][rank], (uint32_t)lane);
           const uint32_t rb = peer_addr(&tl->rbar[slot], (uint32_t)lane);
-          st_async_v4(ra, mT, sT, mD, sD, rb);
-          st_async_v4(ra + 16, zxT, zxD, want_tv ? tvp : 0.f, 0.f, rb);
+          st_async_v4(ra, mT, sumT, mD, sumD, rb);
+          st_async_v4(ra + 16, zxT, zxD, 0.f, 0.f, rb);
         }
-      } else {
-        tvp = warp_sum(tvp);
-        if (want_tv && nrows > 0) {  // final iteration: the last row's TV goes to the leader
-          if (leader && lane == 0) mbar_arrive_expect_tx(&tl->fbar, C * 4u);
-          if (lane == 0)
-            st_async_b32(peer_addr(&tl->frecv[rank], 0), __float_as_uint(tvp), peer_addr(&tl->fbar, 0));
-        }
+        if (++stage == nS) stage = 0;
       }
-      if (it > 0 && ((it - 1) % a.R) == a.K) {  // row it-1's bonus candidate goes to the leader
-        const int pslot = (it - 1) % kRing;
-        Cand c2 = lane < nwarps ? tl->wcand[par][lane] : cand_empty();
-        c2 = warp_cand(c2);
-        if (leader && lane == 0) mbar_arrive_expect_tx(&tl->cbar[pslot], C * (uint32_t)sizeof(Cand));
+      if (it >= 1) {  // row it-1: phase B done in this CTA
+        const int p = it - 1;
+        swait(&tl->bfull[p & 1], (uint32_t)((p >> 1) & 1), tl, a.dev_err, kWsBfull);
+        float tv = lane < nwarps ? tl->wtv[p & 1][lane] : 0.f;
+        tv = warp_sum(tv);
+        const int pk = k == 0 ? a.R - 1 : k - 1;
+        Cand cd = cand_empty();
+        if (pk == a.K) {
+          if (lane < nwarps) cd = tl->wcand[p & 1][lane];
+          cd = warp_cand(cd);
+        }
+        const int pslot = p % kRing;
+        if (leader && lane == 0) mbar_arrive_expect_tx(&tl->bbar[pslot], C * (uint32_t)sizeof(BMsg));
         if (lane == 0) {
-          const uint32_t ra = peer_addr(&tl->crecv[pslot][rank], 0);
-          const uint32_t rb = peer_addr(&tl->cbar[pslot], 0);
-          st_async_v4(ra, c2.s, c2.lo, c2.hi, c2.ohi, rb);
-          st_async_v4(ra + 16, __int_as_float(c2.idx), 0.f, 0.f, 0.f, rb);
+          const uint32_t ra = peer_addr(&tl->brecv[pslot][rank], 0);
+          const uint32_t rb = peer_addr(&tl->bbar[pslot], 0);
+          st_async_v4(ra, want_tv ? tv : 0.f, cd.s, cd.lo, cd.hi, rb);
+          st_async_v4(ra + 16, cd.ohi, __int_as_float(cd.idx), 0.f, 0.f, rb);
         }
       }
-      if (++k == a.R) k = 0;
+      if (it < nrows && ++k == a.R) k = 0;
     }
+    // Every bulk copy this warp issued has landed before the CTA may exit (they
+    // all have, unless a wait gave up above).
+    if (lane == 0)
+      for (int st = 0; st < nS && st < nrows; ++st)
+        mbar_wait(&tl->full[st], (uint32_t)(((nrows - 1 - st) / nS) & 1));
     cluster_sync();
+    tmem_fence_after();
+    tmem_dealloc(tl->tmem_base, kTmemCols);
     return;
   }
 
   // ---------------- compute warps
-  float xt[EPT], xd[EPT], dp[EPT];
+  // TMEM columns of this warp: lanes 32 * (warp % 4) .., 128 columns from
+  // 128 * (warp / 4): two row buffers of 64 (32 target exps, then 32 draft exps).
+  const uint32_t tcol = tl->tmem_base + ((32u * (uint32_t)(warp & 3)) << 16) + 128u * (uint32_t)(warp >> 2);
   float mwT_p = 0.f, mwD_p = 0.f;  // previous row's warp maxima (safe forms)
   bool okT_p = false, okD_p = false;
-  const float inv_tau = a.inv_tau;
-  int k = 0;          // position of row `it` within its particle
-  int64_t unit = cid; // particle of row `it`
+  int k = 0;           // position of row `it` within its particle
+  int64_t unit = cid;  // particle of row `it`
+  int stage = 0;
+  uint32_t phase = 0;
+  const float cT = a.cT;
   int x_next = (nrows > 0 && a.K > 0) ? a.draft[(int64_t)cid * a.K] : -1;
 
   for (int it = 0; it <= nrows; ++it) {
     const bool cur = it < nrows;
-    const bool prev = it > 0;
-    const int par = it & 1;
     const int x = (cur && k < a.K) ? x_next : -1;
     {  // prefetch the draft token of row it+1
       int kn = k + 1;
@@ -1439,107 +1598,167 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
       x_next = (it + 1 < nrows && kn < a.K) ? a.draft[un * a.K + kn] : -1;
     }
 
-    // ---- previous row: normalisers, bonus screen (only the pending draft exps are live)
-    float scT = 0.f, scD = 0.f;
-    if (prev) {
-      const int pit = it - 1;
-      const int pslot = pit % kRing;
+    // ---------------- phase A: row it
+    float mwTs = 0.f, mwDs = 0.f;
+    bool okT = false, okD = false;
+    if (cur) {
+      swait(&tl->full[stage], phase, tl, a.dev_err, kWsFull);
+      const int64_t row = unit * a.R + k;
+      const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb);
+      const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb + sb);
+      const TIn* gT = (const TIn*)a.zT + row * a.ld + s0;
+      const TIn* gD = (const TIn*)a.zD + row * a.ld + s0;
+      // pass 1: maxima
+      uint4 rT[HOLD ? CPT : 1], rD[HOLD ? CPT : 1];
+      typename CK::Acc aT = CK::kAcc0, aD = CK::kAcc0;
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        const int e0 = (tid + c * ncomp) * EPC;
+        const uint4 vT = load_chunk<TIn>(stT, gT, e0, len, tma_len);
+        const uint4 vD = load_chunk<TIn>(stD, gD, e0, len, tma_len);
+        CK::max_acc(aT, vT);
+        CK::max_acc(aD, vD);
+        if (HOLD) {
+          rT[HOLD ? c : 0] = vT;
+          rD[HOLD ? c : 0] = vD;
+        }
+      }
+      if (x >= s0 && x < s0 + len) {  // the owner of the draft token records its raw logits
+        const int le = x - s0;
+        if (((le / EPC) % ncomp) == tid) {
+          tl->zx[it & 1][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
+          tl->zx[it & 1][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
+        }
+      }
+      float mwT = CK::acc_f32(aT), mwD = CK::acc_f32(aD);
+      warp_max2_nan(mwT, mwD);
+      okT = mwT > -INFINITY;
+      okD = mwD > -INFINITY;
+      mwTs = mwT == -INFINITY ? 0.f : mwT;
+      mwDs = mwD == -INFINITY ? 0.f : mwD;
+      // pass 2: e = 2^(z cT - m cT) for both halves, summed and parked in TMEM
+      const float2 c2 = f2(cT), nT2 = f2(-mwTs * cT), nD2 = f2(-mwDs * cT);
+      const uint32_t tb = tcol + 64u * (uint32_t)(it & 1);
+      float2 accT = f2(0.f), accD = f2(0.f);
+      float eT[8], eD[8];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        uint4 vT, vD;
+        if (HOLD) {
+          vT = rT[HOLD ? c : 0];
+          vD = rD[HOLD ? c : 0];
+        } else {
+          const int e0 = (tid + c * ncomp) * EPC;
+          vT = load_chunk<TIn>(stT, gT, e0, len, tma_len);
+          vD = load_chunk<TIn>(stD, gD, e0, len, tma_len);
+        }
+#pragma unroll
+        for (int j = 0; j < EPC; j += 2) {
+          const int i = (c * EPC + j) & 7;
+          const float2 tT = __ffma2_rn(make_float2(CK::elem(vT, j), CK::elem(vT, j + 1)), c2, nT2);
+          const float2 tD = __ffma2_rn(make_float2(CK::elem(vD, j), CK::elem(vD, j + 1)), c2, nD2);
+          eT[i] = ex2(tT.x);
+          eT[i + 1] = ex2(tT.y);
+          eD[i] = ex2(tD.x);
+          eD[i + 1] = ex2(tD.y);
+          accT = __fadd2_rn(accT, make_float2(eT[i], eT[i + 1]));
+          accD = __fadd2_rn(accD, make_float2(eD[i], eD[i + 1]));
+          if (i + 2 == 8) {  // eight entries done: park them (whole warp, converged)
+            const uint32_t col = (uint32_t)((c * EPC + j + 2) - 8);
+            __syncwarp();
+            tmem_st8(tb + col, eT);
+            tmem_st8(tb + 32u + col, eD);
+          }
+        }
+      }
+      float sTw = accT.x + accT.y, sDw = accD.x + accD.y;
+      warp_sum2(sTw, sDw);
+      if (lane == 0) tl->wpart[it & 1][warp] = make_float4(mwT, sTw, mwD, sDw);
+      __syncwarp();
+      tmem_wait_st();
+      // all compute warps are done with row it (and its stage): one arrival
+      bar_sync_n(1, ncomp);
+      if (warp == 0 && lane == 0) mbar_arrive(&tl->afull[it & 1]);
+    }
+
+    // ---------------- phase B: row it-1
+    if (it > 0) {
+      const int p = it - 1;
+      const int pslot = p % kRing;
       const int pk = k == 0 ? a.R - 1 : k - 1;
       const int64_t punit = k == 0 ? unit - G : unit;
-      if (!mbar_wait(&tl->rbar[pslot], (uint32_t)((pit / kRing) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
+      swait(&tl->rbar[pslot], (uint32_t)((p / kRing) & 1), tl, a.dev_err, kWsRow);
       const Msg* rv = tl->recv[pslot];
       const bool has = lane < (int)C;
       const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
-                               has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, a.cT);
-      scT = (!nm.badT && okT_p) ? ex2((mwT_p - nm.MT) * a.cT) / nm.ST : 0.f;
-      scD = (!nm.badD && okD_p) ? ex2((mwD_p - nm.MD) * a.cT) / nm.SD : 0.f;
-      if (pk == a.K) {
-        Cand cd = cand_empty();
-        if (!nm.badT && okT_p) {
-          // Tref = M/tau + g_min - margin: a lower bound on the winning score.
-          const float margin = 1e-5f + 2e-7f * fabsf(nm.MT * inv_tau);
-          const float rho = ex2((mwT_p - nm.MT) * a.cT + (-kGumbelMinF + margin) * kLog2e);
-          const float mw_a = mwT_p * inv_tau;
-          const Stream st(a.seed, a.round, SD_STREAM_BONUS);
+                               has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, cT);
+      const bool gT_ok = !nm.badT && okT_p, gD_ok = !nm.badD && okD_p;
+      const float scT = gT_ok ? ex2((mwT_p - nm.MT) * cT) / nm.ST : 0.f;
+      const float scD = gD_ok ? ex2((mwD_p - nm.MD) * cT) / nm.SD : 0.f;
+      const bool bonus = pk == a.K;
+      const uint32_t tb = tcol + 64u * (uint32_t)(p & 1);
+      float eT[kEPT], eD[kEPT];
+      __syncwarp();  // the lanes left the wait above one by one
 #pragma unroll
-          for (int q = 0; q < EPT / 4; ++q) {
-            const int c = q / (EPC / 4);
-            const int e0 = (tid + c * ncomp) * EPC + (q % (EPC / 4)) * 4;
-            if (e0 >= len) continue;
-            const float4 ev = tbuf[q * ncomp + tid];
-            const float y0 = ev.x * rho, y1 = ev.y * rho, y2 = ev.z * rho, y3 = ev.w * rho;
-            if (fmaxf(fmaxf(y0, y1), fmaxf(y2, y3)) < kYSkip) continue;
-            const int v0 = s0 + e0;
-            const U4 w = st.at((uint32_t)(v0 >> 2), (uint32_t)punit);
-            const float u0 = uniform_f32(w.x), u1 = uniform_f32(w.y);
-            const float u2 = uniform_f32(w.z), u3 = uniform_f32(w.w);
-            const bool k0 = keep_bonus(y0, u0) && e0 + 0 < len;
-            const bool k1 = keep_bonus(y1, u1) && e0 + 1 < len;
-            const bool k2 = keep_bonus(y2, u2) && e0 + 2 < len;
-            const bool k3 = keep_bonus(y3, u3) && e0 + 3 < len;
-            if (k0 | k1 | k2 | k3) {
-              if (k0) cd = cand_merge(cd, bonus_cand(ev.x, u0, mw_a, v0));
-              if (k1) cd = cand_merge(cd, bonus_cand(ev.y, u1, mw_a, v0 + 1));
-              if (k2) cd = cand_merge(cd, bonus_cand(ev.z, u2, mw_a, v0 + 2));
-              if (k3) cd = cand_merge(cd, bonus_cand(ev.w, u3, mw_a, v0 + 3));
-            }
-          }
-        }
-        cd = warp_cand(cd);
-        if (lane == 0) tl->wcand[par][warp] = cd;
+      for (int i = 0; i < kEPT; i += 8) {
+        tmem_ld8(tb + (uint32_t)i, &eT[i]);
+        tmem_ld8(tb + 32u + (uint32_t)i, &eD[i]);
       }
+      tmem_wait_ld();
+      float tvw;
+      Cand cd = cand_empty();
+      if (scT > 0.f) {
+        // sum |p - q| = scT * sum |eT - eD * (scD / scT)|: one fused op per entry,
+        // exactly 0 for identical rows (ratio 1).
+        const float2 nr2 = f2(-(scD / scT));
+        float2 t2 = f2(0.f);
+#pragma unroll
+        for (int i = 0; i < kEPT; i += 2) {
+          const float2 d = __ffma2_rn(make_float2(eD[i], eD[i + 1]), nr2, make_float2(eT[i], eT[i + 1]));
+          t2 = __fadd2_rn(t2, make_float2(fabsf(d.x), fabsf(d.y)));
+        }
+        tvw = scT * (t2.x + t2.y);
+        if (bonus) {
+          // Tref = M/tau + g_min - margin bounds the winning score from below
+          const float margin = 1e-5f + 2e-7f * fabsf(nm.MT * a.inv_tau);
+          const float rho = ex2((mwT_p - nm.MT) * cT + (-kGumbelMinF + margin) * kLog2e);
+          const TIn* gT = (const TIn*)a.zT + (punit * a.R + pk) * a.ld + s0;
+          cd = bonus_screen<TIn>(tb, gT, s0, len, tid, ncomp, rho, a.inv_tau,
+                                 Stream(a.seed, a.round, SD_STREAM_BONUS), (uint32_t)punit);
+        }
+      } else {  // no target mass in this warp's entries (or a bad row): TV part = sum q
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kEPT; ++i) s += eD[i];
+        tvw = scD * s;
+      }
+      tvw = warp_sum(tvw);
+      if (bonus) cd = warp_cand(cd);
+      if (lane == 0) {
+        tl->wtv[p & 1][warp] = tvw;
+        if (bonus) tl->wcand[p & 1][warp] = cd;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->bfull[p & 1]);
     }
 
-    // ---- current row: ring -> registers, maxima
-    float mwT = -INFINITY, mwD = -INFINITY;
     if (cur) {
-      if (!mbar_wait(&tl->full[par], (uint32_t)((it >> 1) & 1))) raise_err(a.dev_err, SD_DEV_TIMEOUT);
-      const int64_t row = unit * a.R + k;
-      const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes);
-      const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)par * 2 * a.stage_bytes + a.stage_bytes);
-      const TIn* gT = (const TIn*)a.zT + row * a.ld + s0;
-      const TIn* gD = (const TIn*)a.zD + row * a.ld + s0;
-      mwT = load_slice<TIn, CPT>(xt, stT, gT, len, tma_len, tid, ncomp);
-      mwD = load_slice<TIn, CPT>(xd, stD, gD, len, tma_len, tid, ncomp);
-      if (x >= s0 && x < s0 + len) {
-        const int le = x - s0;
-        if (((le / EPC) % ncomp) == tid) {
-          tl->zx[par][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
-          tl->zx[par][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
-        }
+      mwT_p = mwTs;
+      mwD_p = mwDs;
+      okT_p = okT;
+      okD_p = okD;
+      if (++stage == nS) {
+        stage = 0;
+        phase ^= 1u;
       }
-      warp_max2(mwT, mwD);
-    }
-    const float mwTs = mwT == -INFINITY ? 0.f : mwT;
-    const float mwDs = mwD == -INFINITY ? 0.f : mwD;
-
-    // ---- fused pass: row r exps + row r-1 TV ----
-    float sT = 0.f, sD = 0.f, tv = 0.f;
-    if (cur && prev)
-      fused_pass<CPT, EPC, true, true>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD, sT,
-                                       sD, tv);
-    else if (cur)
-      fused_pass<CPT, EPC, true, false>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD,
-                                        sT, sD, tv);
-    else if (prev)
-      fused_pass<CPT, EPC, false, true>(xt, xd, dp, tbuf, tid, ncomp, mwTs, mwDs, a.cT, scT, scD,
-                                        sT, sD, tv);
-    warp_sum3(sT, sD, tv);
-    if (lane == 0) {
-      tl->wpart[par][warp] = make_float4(mwT, sT, mwD, sD);
-      tl->tvw[par][warp] = tv;
-    }
-    // (A) post this iteration's partials to the communication warp and move on
-    asm volatile("bar.arrive 1, %0;" ::"r"(ncomp + 32) : "memory");
-    mwT_p = mwTs;
-    mwD_p = mwDs;
-    okT_p = mwT > -INFINITY;
-    okD_p = mwD > -INFINITY;
-    if (cur && ++k == a.R) {
-      k = 0;
-      unit += G;
+      if (++k == a.R) {
+        k = 0;
+        unit += G;
+      }
     }
   }
+  __syncwarp();
+  tmem_fence_before();
   cluster_sync();
 }
 
@@ -1641,8 +1860,12 @@ static bool make_plan(const void* fn, int V, int esize, int64_t units, LaunchPla
   return found;
 }
 
-// Launch plan of the pipelined SMC-SD kernel: one warp group per CTA, two
-// ring stages, plus the target-exps buffer (32 fp32 per compute thread).
+// Launch plan of the pipelined SMC-SD kernel: one compute warp group per CTA
+// (32 entries per thread per row, at most 16 warps so that two TMEM row buffers
+// per warp fit) plus the communication and bookkeeping warps; the deepest ring
+// that fits, and at least kMinSmem of shared memory so that one CTA runs per
+// SM (it takes all of the SM's tensor memory).  Among the cluster sizes it
+// keeps the most SMs busy for this many particles.
 static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, LaunchPlan& best) {
   static std::mutex mu;
   static std::map<std::tuple<const void*, int, int, int, int64_t>, LaunchPlan> cache;
@@ -1666,14 +1889,20 @@ static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, Launc
     const int threads = ncomp + 64;  // + communication and bookkeeping warps
     if (threads > kMaxThreads || ncomp / 32 > kMaxWarps) continue;
     const uint32_t sb = (uint32_t)(((int64_t)slice * esize + 127) / 128 * 128);
-    const size_t smem = (size_t)2 * 2 * sb + (size_t)ncomp * kEPT * 4 + sizeof(SmcTail) + 128;
-    if (smem > (size_t)optin) continue;
+    int nS = 0;
+    for (int st = kMaxStages; st >= 2; --st)
+      if ((size_t)st * 2 * sb + sizeof(SmcTail) + 128 <= (size_t)optin) {
+        nS = st;
+        break;
+      }
+    if (nS == 0) continue;
+    const size_t smem = std::max((size_t)nS * 2 * sb + sizeof(SmcTail) + 128, kMinSmem);
     const int nc = max_active_clusters(fn, C, threads, smem);
     if (nc <= 0) continue;
-    const int64_t score = std::min<int64_t>(ukey, nc) * C;
+    const int64_t score = std::min<int64_t>(ukey, nc) * C * 8 + nS;
     if (score > best_score) {
       best_score = score;
-      best = LaunchPlan{C, 1, threads, 2, slice, sb, smem, nc};
+      best = LaunchPlan{C, 1, threads, nS, slice, sb, smem, nc};
       found = true;
     }
   }
@@ -1686,12 +1915,12 @@ static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, Launc
 
 template <typename TIn>
 static sd_status launch_smc(ScoreArgs& a, cudaStream_t stream) {
-  const void* fn = (const void*)smc_kernel<TIn, (int)(kEPT * sizeof(TIn) / 16)>;
+  const void* fn = (const void*)smc_kernel<TIn>;
   LaunchPlan p;
   if (!make_plan_smc(fn, a.V, (int)sizeof(TIn), a.units, p)) return SD_ERR_UNSUPPORTED;
   a.slice = p.slice;
   a.groups = 1;
-  a.stages = 2;
+  a.stages = p.stages;
   a.stage_bytes = p.stage_bytes;
   const bool aligned = ((uintptr_t)a.zT % 16 == 0) && ((uintptr_t)a.zD % 16 == 0) &&
                        ((a.ld * (int64_t)sizeof(TIn)) % 16 == 0);
@@ -1714,7 +1943,8 @@ static sd_status launch_smc(ScoreArgs& a, cudaStream_t stream) {
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, smc_kernel<TIn, (int)(kEPT * sizeof(TIn) / 16)>, a);
+  void* args[] = {(void*)&a};
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return SD_ERR_CUDA;

@@ -57,7 +57,7 @@ struct ScoreArgs {
   uint32_t stage_bytes;  // bytes reserved for one tensor's slice in a stage
   int use_tma;
   float inv_tau, cT;     // 1/tau and log2(e)/tau, fp32
-  double tau64;
+  double tau64, inv_tau64;
   const int32_t* draft;  // [units, K]
   uint64_t seed, round;
   const double* logw_prev;
@@ -1033,30 +1033,31 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
 // the last row of each particle also draws the bonus token.  A cluster of C
 // CTAs walks its particles' rows in order; CTA r owns vocabulary slice r.
 //
-// Iteration `it` of the compute warps has two phases:
-//   A(it)    row it: move its slices from the ring to registers, warp maxima,
-//            exps (one MUFU exp2 per entry) and sums; the exps of both halves
-//            go to tensor memory (TMEM), two row buffers per warp.  The
-//            compute warps then meet at one barrier and post their (max, sum)
-//            partials.
-//   B(it-1)  row it-1: wait for its messages from the cluster (sent during
-//            phase A, so the exchange is hidden behind it), rebuild the row
-//            normalisers, read the row's exps back from TMEM and take the TV
-//            partial sum |p - q|; on a particle's last row also screen the
-//            bonus-token candidates.
-// A communication warp turns the warp partials into one 32-byte message per
-// row for every CTA of the cluster (st.async into distributed shared memory,
-// completing on the receiver's mbarrier -- no cluster barrier on the row
-// path), sends each row's TV partial and bonus candidate to the leader, and
-// refills the ring with bulk async copies (no multicast) once phase A has
-// released a stage.  The leader's bookkeeping warp turns the messages into
-// fp64 lse, log-probs, log-weights, TV and bonus tokens (near-ties settled
-// exactly in fp64).  Every element is read from HBM once and exponentiated once.
+// Warp roles of a CTA:
+//   producers (one per 32 x 32 entries of the slice), row by row: move the
+//     row's slices from the ring to registers, warp maxima, exps (one MUFU
+//     exp2 per entry) and sums; the exps of both halves go to tensor memory
+//     (TMEM, two row buffers per warp); post the (max, sum) partials.
+//   consumers (four, one per TMEM lane quarter), one row behind: once the
+//     row's messages are in, rebuild its normalisers, read the exps back from
+//     TMEM and take the TV partial sum |p - q|; on a particle's last row also
+//     screen the bonus-token candidates; then hand the row buffer back.
+//   communication: turns the producers' partials into one 32-byte message per
+//     row for every CTA of the cluster (st.async into distributed shared
+//     memory, completing on the receiver's mbarrier -- no cluster barrier on
+//     the row path), sends each row's TV partial and bonus candidate to the
+//     leader, and refills the ring with bulk async copies (no multicast).
+//   bookkeeping (leader only): fp64 lse, log-probs, log-weights, TV and bonus
+//     tokens (near-ties settled exactly in fp64).
+// MUFU work (producers) and the exchange plus TV (consumers) overlap; every
+// element is read from HBM once and exponentiated once.
 
 constexpr int kRing = 8;     // message slots per CTA
 constexpr int kLead = 2;     // rows a CTA's messages can run ahead of the leader's
 constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 512;  // all of the SM's tensor memory (one CTA per SM)
+constexpr int kConsumers = 4;        // phase-B warps, one per TMEM lane quarter
+constexpr int kMaxThreadsSmc = 640;  // up to 14 producers + 4 consumers + 2 service warps
 constexpr size_t kMinSmem = 120 * 1024;  // > half an SM's shared memory: one CTA per SM
 
 struct alignas(16) BMsg {  // one slice's phase-B results for the leader
@@ -1068,15 +1069,18 @@ struct alignas(16) BMsg {  // one slice's phase-B results for the leader
 
 struct alignas(128) SmcTail {
   uint64_t full[kMaxStages];    // ring stages (target and draft slices of one row)
-  uint64_t afull[2], bfull[2];  // compute warps -> communication warp, by row parity
+  uint64_t afull[2];  // producers done with a row (exps in TMEM, partials posted)
+  uint64_t bfull[2];  // consumers done with a row (TV partials, candidates posted)
+  uint64_t tfree[2];  // consumers done reading a TMEM row buffer
+  uint64_t sfin;      // producers posted the last row's bonus candidates
   uint64_t rbar[kRing], bbar[kRing], adone[kRing];
   int abort_flag;
   uint32_t tmem_base;
   Msg recv[kRing][kMaxCluster];
   BMsg brecv[kRing][kMaxCluster];
   float4 wpart[2][kMaxWarps];
-  float wtv[2][kMaxWarps];
-  Cand wcand[2][kMaxWarps];
+  float wtv[2][kConsumers];
+  Cand wcand[4][kMaxWarps];  // producers' bonus candidates, by row & 3
   float zx[2][2];
 };
 
@@ -1128,12 +1132,24 @@ __device__ __forceinline__ void warp_sum2(float& a, float& b) {
     b += y;
   }
 }
-// fp64 lse of a row from per-slice partials (one per lane, `has` marks valid
-// lanes); the slice factors use MUFU exp2, the sum and the log are fp64.
-__device__ __noinline__ double row_lse_fast(float m, float s, float M, bool has, double tau64,
-                                            float cT) {
-  const double t = (has && m > -INFINITY) ? (double)s * (double)ex2((m - M) * cT) : 0.0;
-  return (double)M / tau64 + log(warp_sum_d(t));
+// fp64 lse of a row's target and draft halves from the C slice partials of its
+// messages: half-warp 0 sums the target's, half-warp 1 the draft's, and both
+// logs run at once.  Slice factors use MUFU exp2, the sums and logs are fp64.
+struct Lse2 {
+  double T, D;
+};
+__device__ __noinline__ Lse2 row_lse_pair(const Msg* e, uint32_t C, float MT, float MD,
+                                          double inv_tau64, float cT) {
+  const int lane = threadIdx.x & 31, h = lane >> 4, l = lane & 15;
+  const bool has = l < (int)C;
+  const float m = has ? (h ? e[l].mD : e[l].mT) : -INFINITY;
+  const float s = has ? (h ? e[l].sD : e[l].sT) : 0.f;
+  const float M = h ? MD : MT;
+  double t = m > -INFINITY ? (double)s * (double)ex2((m - M) * cT) : 0.0;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  const double lse = (double)M * inv_tau64 + log(t);
+  return Lse2{__shfl_sync(0xffffffffu, lse, 0), __shfl_sync(0xffffffffu, lse, 16)};
 }
 
 // Row normalisers from per-slice (max, sum) partials held one per lane.  A
@@ -1345,10 +1361,8 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
       const bool has = lane < (int)C;
       const Norm nm = row_norm(has ? e[lane].mT : -INFINITY, has ? e[lane].sT : 0.f,
                                has ? e[lane].mD : -INFINITY, has ? e[lane].sD : 0.f, a.cT);
-      const double lse64T = row_lse_fast(has ? e[lane].mT : -INFINITY, has ? e[lane].sT : 0.f,
-                                         nm.MT, has, a.tau64, a.cT);
-      const double lse64D = row_lse_fast(has ? e[lane].mD : -INFINITY, has ? e[lane].sD : 0.f,
-                                         nm.MD, has, a.tau64, a.cT);
+      const Lse2 lse = row_lse_pair(e, C, nm.MT, nm.MD, a.inv_tau64, a.cT);
+      const double lse64T = lse.T, lse64D = lse.D;
       bad_cur = nm.badT || nm.badD;
       badT_cur = nm.badT;
       int x = -1;
@@ -1374,8 +1388,8 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
           double lp = NAN, lq = NAN;
           if (!x_ok) raise_err(a.dev_err, SD_DEV_TOKEN_OOB);
           if (x_ok && !bad_cur) {
-            lp = (double)zxT / a.tau64 - lse64T;
-            lq = (double)zxD / a.tau64 - lse64D;
+            lp = (double)zxT * a.inv_tau64 - lse64T;
+            lq = (double)zxD * a.inv_tau64 - lse64D;
           } else {
             unit_bad = true;
           }
@@ -1439,16 +1453,18 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs a) {
   using CK = Chunk<TIn>;
   constexpr int EPC = CK::EPC;
-  constexpr int CPT = kEPT / EPC;          // chunks per thread
+  constexpr int CPT = kEPT / EPC;          // chunks per producer thread
   constexpr bool HOLD = sizeof(TIn) == 2;  // bf16: raw chunks stay in registers for pass 2
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // warps [0, nwarps): compute; warp nwarps: communication; warp nwarps+1: bookkeeping
-  const int ncomp = blockDim.x - 64, nwarps = ncomp >> 5;
+  // warps [0, nA): producers; [nA, nA + 4): consumers; then communication, bookkeeping
+  const int nA = (int)(blockDim.x >> 5) - kConsumers - 2;
+  const int ncomp = nA * 32;
+  const int wComm = nA + kConsumers, wBook = wComm + 1;
   const uint32_t rank = cluster_rank(), C = cluster_size();
   const uint32_t cid = cluster_id(), G = num_clusters();
   const int nS = a.stages;
@@ -1463,13 +1479,16 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
   const int nrows = (int)(my_units * a.R);
   const bool leader = rank == 0;
   const bool want_tv = a.tv_out != nullptr;
+  const float cT = a.cT;
 
   if (tid == 0) {
     for (int st = 0; st < nS; ++st) mbar_init(&tl->full[st], 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&tl->afull[b], 1);
-      mbar_init(&tl->bfull[b], (uint32_t)nwarps);
+      mbar_init(&tl->afull[b], (uint32_t)nA);
+      mbar_init(&tl->bfull[b], kConsumers);
+      mbar_init(&tl->tfree[b], kConsumers);
     }
+    mbar_init(&tl->sfin, (uint32_t)nA);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&tl->rbar[i], 1);
       mbar_init(&tl->bbar[i], 1);
@@ -1478,7 +1497,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
     tl->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == nwarps) {  // the communication warp owns the CTA's tensor memory
+  if (warp == wComm) {  // the communication warp owns the CTA's tensor memory
     tmem_alloc(&tl->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -1487,13 +1506,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
   tmem_fence_after();
   cluster_sync();
 
-  if (warp == nwarps + 1) {  // ---------------- bookkeeping (leader only)
+  if (warp == wBook) {  // ---------------- bookkeeping (leader only)
     if (leader) smc_bookkeep<TIn>(a, tl, C, cid, G, nrows, want_tv);
     cluster_sync();
     return;
   }
 
-  if (warp == nwarps) {  // ---------------- communication warp
+  if (warp == wComm) {  // ---------------- communication warp
     const uint64_t pol = policy_evict_first();
     // stage st <- row `it` of this cluster: unit cid + (it / R) * G, position it % R
     auto issue = [&](int it, int st) {
@@ -1509,14 +1528,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
       for (int i = 0; i < nS && i < nrows; ++i) issue(i, i);
     int k = 0, stage = 0;  // position and ring stage of row it
     for (int it = 0; it <= nrows; ++it) {
-      if (it < nrows) {  // row it: phase A done in this CTA; its stage is free
+      if (it < nrows) {  // row it: the producers are done with it and with its stage
         swait(&tl->afull[it & 1], (uint32_t)((it >> 1) & 1), tl, a.dev_err, kWsAfull);
         if (lane == 0 && it + nS < nrows) issue(it + nS, stage);
         const float4 wp =
-            lane < nwarps ? tl->wpart[it & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+            lane < nA ? tl->wpart[it & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
         float mT = wp.x, mD = wp.z;
         warp_max2_nan(mT, mD);  // a warp's NaN max (NaN in its entries) must reach the sum
-        float sumT = part_term(wp.x, wp.y, mT, a.cT), sumD = part_term(wp.z, wp.w, mD, a.cT);
+        float sumT = part_term(wp.x, wp.y, mT, cT), sumD = part_term(wp.z, wp.w, mD, cT);
         warp_sum2(sumT, sumD);
         float zxT = 0.f, zxD = 0.f;
         if (k < a.K) {
@@ -1539,15 +1558,16 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
         }
         if (++stage == nS) stage = 0;
       }
-      if (it >= 1) {  // row it-1: phase B done in this CTA
+      if (it >= 1) {  // row it-1: the consumers are done with it
         const int p = it - 1;
         swait(&tl->bfull[p & 1], (uint32_t)((p >> 1) & 1), tl, a.dev_err, kWsBfull);
-        float tv = lane < nwarps ? tl->wtv[p & 1][lane] : 0.f;
+        float tv = lane < kConsumers ? tl->wtv[p & 1][lane] : 0.f;
         tv = warp_sum(tv);
         const int pk = k == 0 ? a.R - 1 : k - 1;
         Cand cd = cand_empty();
-        if (pk == a.K) {
-          if (lane < nwarps) cd = tl->wcand[p & 1][lane];
+        if (pk == a.K) {  // the producers screened it during the next row (the last: on its own)
+          if (p == nrows - 1) swait(&tl->sfin, 0u, tl, a.dev_err, kWsBfull);
+          if (lane < nA) cd = tl->wcand[p & 3][lane];
           cd = warp_cand(cd);
         }
         const int pslot = p % kRing;
@@ -1572,22 +1592,107 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
     return;
   }
 
-  // ---------------- compute warps
-  // TMEM columns of this warp: lanes 32 * (warp % 4) .., 128 columns from
-  // 128 * (warp / 4): two row buffers of 64 (32 target exps, then 32 draft exps).
+  if (warp >= nA) {  // ---------------- consumers
+    // Quarter q of TMEM holds the rows of producers q, q + 4, ...: 128 columns
+    // from 128 * (w / 4), two row buffers of 64 (32 target exps, 32 draft exps).
+    const int q = warp & 3, cidx = warp - nA;
+    const uint32_t tq = tl->tmem_base + ((32u * (uint32_t)q) << 16);
+    for (int p = 0; p < nrows; ++p) {
+      swait(&tl->afull[p & 1], (uint32_t)((p >> 1) & 1), tl, a.dev_err, kWsAfull);
+      swait(&tl->rbar[p % kRing], (uint32_t)((p / kRing) & 1), tl, a.dev_err, kWsRow);
+      __syncwarp();
+      tmem_fence_after();
+      const Msg* rv = tl->recv[p % kRing];
+      const bool has = lane < (int)C;
+      const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
+                               has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, cT);
+      float tv = 0.f;
+      for (int w = q; w < nA; w += 4) {
+        const float4 wp = tl->wpart[p & 1][w];  // producer w's raw maxima and sums
+        const float scT = (!nm.badT && wp.x > -INFINITY) ? ex2((wp.x - nm.MT) * cT) / nm.ST : 0.f;
+        const float scD = (!nm.badD && wp.z > -INFINITY) ? ex2((wp.z - nm.MD) * cT) / nm.SD : 0.f;
+        const uint32_t tb = tq + 128u * (uint32_t)(w >> 2) + 64u * (uint32_t)(p & 1);
+        if (scT > 0.f) {
+          // sum |p - q| = scT * sum |eT - eD * (scD / scT)|: one fused op per entry,
+          // exactly 0 for identical rows (ratio 1).
+          const float2 nr2 = f2(-(scD / scT));
+          float2 t2 = f2(0.f);
+#pragma unroll
+          for (int i = 0; i < kEPT; i += 16) {
+            float eT[16], eD[16];
+            tmem_ld8(tb + (uint32_t)i, &eT[0]);
+            tmem_ld8(tb + (uint32_t)i + 8u, &eT[8]);
+            tmem_ld8(tb + 32u + (uint32_t)i, &eD[0]);
+            tmem_ld8(tb + 40u + (uint32_t)i, &eD[8]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+              const float2 d = __ffma2_rn(make_float2(eD[j], eD[j + 1]), nr2, make_float2(eT[j], eT[j + 1]));
+              t2 = __fadd2_rn(t2, make_float2(fabsf(d.x), fabsf(d.y)));
+            }
+          }
+          tv += scT * (t2.x + t2.y);
+        } else if (scD > 0.f) {  // no target mass in these entries (or a bad row): TV part = sum q
+          float sq = 0.f;
+#pragma unroll
+          for (int i = 0; i < kEPT; i += 8) {
+            float eD[8];
+            tmem_ld8(tb + 32u + (uint32_t)i, eD);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) sq += eD[j];
+          }
+          tv += scD * sq;
+        }
+      }
+      // the row buffer goes back to the producers
+      __syncwarp();
+      tmem_fence_before();
+      if (lane == 0) mbar_arrive(&tl->tfree[p & 1]);
+      tv = warp_sum(tv);
+      if (lane == 0) tl->wtv[p & 1][cidx] = tv;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->bfull[p & 1]);
+    }
+    __syncwarp();
+    tmem_fence_before();
+    cluster_sync();
+    return;
+  }
+
+  // ---------------- producers
   const uint32_t tcol = tl->tmem_base + ((32u * (uint32_t)(warp & 3)) << 16) + 128u * (uint32_t)(warp >> 2);
-  float mwT_p = 0.f, mwD_p = 0.f;  // previous row's warp maxima (safe forms)
-  bool okT_p = false, okD_p = false;
   int k = 0;           // position of row `it` within its particle
   int64_t unit = cid;  // particle of row `it`
   int stage = 0;
   uint32_t phase = 0;
-  const float cT = a.cT;
   int x_next = (nrows > 0 && a.K > 0) ? a.draft[(int64_t)cid * a.K] : -1;
+  float mwT_prev = -INFINITY;  // this warp's raw target max of the previous row
 
-  for (int it = 0; it <= nrows; ++it) {
-    const bool cur = it < nrows;
-    const int x = (cur && k < a.K) ? x_next : -1;
+  // Bonus-token screen of row p (a particle's last row) over this warp's entries,
+  // from its exps still in TMEM, once the row's messages give its max M.
+  auto screen = [&](int p, int64_t punit) {
+    swait(&tl->rbar[p % kRing], (uint32_t)((p / kRing) & 1), tl, a.dev_err, kWsRow);
+    __syncwarp();
+    const Msg* rv = tl->recv[p % kRing];
+    const bool has = lane < (int)C;
+    const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
+                             has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, cT);
+    Cand cd = cand_empty();
+    if (!nm.badT && mwT_prev > -INFINITY) {
+      // Tref = M/tau + g_min - margin bounds the winning score from below
+      const float margin = 1e-5f + 2e-7f * fabsf(nm.MT * a.inv_tau);
+      const float rho = ex2((mwT_prev - nm.MT) * cT + (-kGumbelMinF + margin) * kLog2e);
+      const TIn* gT = (const TIn*)a.zT + (punit * a.R + a.K) * a.ld + s0;
+      cd = bonus_screen<TIn>(tcol + 64u * (uint32_t)(p & 1), gT, s0, len, tid, ncomp, rho,
+                             a.inv_tau, Stream(a.seed, a.round, SD_STREAM_BONUS), (uint32_t)punit);
+    }
+    cd = warp_cand(cd);
+    if (lane == 0) tl->wcand[p & 3][warp] = cd;
+  };
+
+  for (int it = 0; it < nrows; ++it) {
+    const int x = k < a.K ? x_next : -1;
     {  // prefetch the draft token of row it+1
       int kn = k + 1;
       int64_t un = unit;
@@ -1597,165 +1702,99 @@ __global__ void __launch_bounds__(kMaxThreads, 1) smc_kernel(const ScoreArgs a) 
       }
       x_next = (it + 1 < nrows && kn < a.K) ? a.draft[un * a.K + kn] : -1;
     }
-
-    // ---------------- phase A: row it
-    float mwTs = 0.f, mwDs = 0.f;
-    bool okT = false, okD = false;
-    if (cur) {
-      swait(&tl->full[stage], phase, tl, a.dev_err, kWsFull);
-      const int64_t row = unit * a.R + k;
-      const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb);
-      const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb + sb);
-      const TIn* gT = (const TIn*)a.zT + row * a.ld + s0;
-      const TIn* gD = (const TIn*)a.zD + row * a.ld + s0;
-      // pass 1: maxima
-      uint4 rT[HOLD ? CPT : 1], rD[HOLD ? CPT : 1];
-      typename CK::Acc aT = CK::kAcc0, aD = CK::kAcc0;
+    swait(&tl->full[stage], phase, tl, a.dev_err, kWsFull);
+    const int64_t row = unit * a.R + k;
+    const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb);
+    const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb + sb);
+    const TIn* gT = (const TIn*)a.zT + row * a.ld + s0;
+    const TIn* gD = (const TIn*)a.zD + row * a.ld + s0;
+    // pass 1: maxima
+    uint4 rT[HOLD ? CPT : 1], rD[HOLD ? CPT : 1];
+    typename CK::Acc aT = CK::kAcc0, aD = CK::kAcc0;
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) {
+    for (int c = 0; c < CPT; ++c) {
+      const int e0 = (tid + c * ncomp) * EPC;
+      const uint4 vT = load_chunk<TIn>(stT, gT, e0, len, tma_len);
+      const uint4 vD = load_chunk<TIn>(stD, gD, e0, len, tma_len);
+      CK::max_acc(aT, vT);
+      CK::max_acc(aD, vD);
+      if (HOLD) {
+        rT[HOLD ? c : 0] = vT;
+        rD[HOLD ? c : 0] = vD;
+      }
+    }
+    if (x >= s0 && x < s0 + len) {  // the owner of the draft token records its raw logits
+      const int le = x - s0;
+      if (((le / EPC) % ncomp) == tid) {
+        tl->zx[it & 1][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
+        tl->zx[it & 1][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
+      }
+    }
+    float mwT = CK::acc_f32(aT), mwD = CK::acc_f32(aD);
+    warp_max2_nan(mwT, mwD);
+    const float mwTs = mwT == -INFINITY ? 0.f : mwT;
+    const float mwDs = mwD == -INFINITY ? 0.f : mwD;
+    // this warp's TMEM row buffer (it & 1) is free once the consumers are done with row it-2
+    if (it >= 2) swait(&tl->tfree[it & 1], (uint32_t)(((it - 2) >> 1) & 1), tl, a.dev_err, kWsRow);
+    __syncwarp();
+    tmem_fence_after();
+    // pass 2: e = 2^(z cT - m cT) for both halves, summed and parked in TMEM
+    const float2 c2 = f2(cT), nT2 = f2(-mwTs * cT), nD2 = f2(-mwDs * cT);
+    const uint32_t tb = tcol + 64u * (uint32_t)(it & 1);
+    float2 accT = f2(0.f), accD = f2(0.f);
+    float eT[8], eD[8];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      uint4 vT, vD;
+      if (HOLD) {
+        vT = rT[HOLD ? c : 0];
+        vD = rD[HOLD ? c : 0];
+      } else {
         const int e0 = (tid + c * ncomp) * EPC;
-        const uint4 vT = load_chunk<TIn>(stT, gT, e0, len, tma_len);
-        const uint4 vD = load_chunk<TIn>(stD, gD, e0, len, tma_len);
-        CK::max_acc(aT, vT);
-        CK::max_acc(aD, vD);
-        if (HOLD) {
-          rT[HOLD ? c : 0] = vT;
-          rD[HOLD ? c : 0] = vD;
-        }
+        vT = load_chunk<TIn>(stT, gT, e0, len, tma_len);
+        vD = load_chunk<TIn>(stD, gD, e0, len, tma_len);
       }
-      if (x >= s0 && x < s0 + len) {  // the owner of the draft token records its raw logits
-        const int le = x - s0;
-        if (((le / EPC) % ncomp) == tid) {
-          tl->zx[it & 1][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
-          tl->zx[it & 1][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
-        }
-      }
-      float mwT = CK::acc_f32(aT), mwD = CK::acc_f32(aD);
-      warp_max2_nan(mwT, mwD);
-      okT = mwT > -INFINITY;
-      okD = mwD > -INFINITY;
-      mwTs = mwT == -INFINITY ? 0.f : mwT;
-      mwDs = mwD == -INFINITY ? 0.f : mwD;
-      // pass 2: e = 2^(z cT - m cT) for both halves, summed and parked in TMEM
-      const float2 c2 = f2(cT), nT2 = f2(-mwTs * cT), nD2 = f2(-mwDs * cT);
-      const uint32_t tb = tcol + 64u * (uint32_t)(it & 1);
-      float2 accT = f2(0.f), accD = f2(0.f);
-      float eT[8], eD[8];
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        uint4 vT, vD;
-        if (HOLD) {
-          vT = rT[HOLD ? c : 0];
-          vD = rD[HOLD ? c : 0];
-        } else {
-          const int e0 = (tid + c * ncomp) * EPC;
-          vT = load_chunk<TIn>(stT, gT, e0, len, tma_len);
-          vD = load_chunk<TIn>(stD, gD, e0, len, tma_len);
+      for (int j = 0; j < EPC; j += 2) {
+        const int i = (c * EPC + j) & 7;
+        const float2 tT = __ffma2_rn(make_float2(CK::elem(vT, j), CK::elem(vT, j + 1)), c2, nT2);
+        const float2 tD = __ffma2_rn(make_float2(CK::elem(vD, j), CK::elem(vD, j + 1)), c2, nD2);
+        eT[i] = ex2(tT.x);
+        eT[i + 1] = ex2(tT.y);
+        eD[i] = ex2(tD.x);
+        eD[i + 1] = ex2(tD.y);
+        accT = __fadd2_rn(accT, make_float2(eT[i], eT[i + 1]));
+        accD = __fadd2_rn(accD, make_float2(eD[i], eD[i + 1]));
+        if (i + 2 == 8) {  // eight entries done: park them (whole warp, converged)
+          const uint32_t col = (uint32_t)((c * EPC + j + 2) - 8);
+          __syncwarp();
+          tmem_st8(tb + col, eT);
+          tmem_st8(tb + 32u + col, eD);
         }
-#pragma unroll
-        for (int j = 0; j < EPC; j += 2) {
-          const int i = (c * EPC + j) & 7;
-          const float2 tT = __ffma2_rn(make_float2(CK::elem(vT, j), CK::elem(vT, j + 1)), c2, nT2);
-          const float2 tD = __ffma2_rn(make_float2(CK::elem(vD, j), CK::elem(vD, j + 1)), c2, nD2);
-          eT[i] = ex2(tT.x);
-          eT[i + 1] = ex2(tT.y);
-          eD[i] = ex2(tD.x);
-          eD[i + 1] = ex2(tD.y);
-          accT = __fadd2_rn(accT, make_float2(eT[i], eT[i + 1]));
-          accD = __fadd2_rn(accD, make_float2(eD[i], eD[i + 1]));
-          if (i + 2 == 8) {  // eight entries done: park them (whole warp, converged)
-            const uint32_t col = (uint32_t)((c * EPC + j + 2) - 8);
-            __syncwarp();
-            tmem_st8(tb + col, eT);
-            tmem_st8(tb + 32u + col, eD);
-          }
-        }
-      }
-      float sTw = accT.x + accT.y, sDw = accD.x + accD.y;
-      warp_sum2(sTw, sDw);
-      if (lane == 0) tl->wpart[it & 1][warp] = make_float4(mwT, sTw, mwD, sDw);
-      __syncwarp();
-      tmem_wait_st();
-      // all compute warps are done with row it (and its stage): one arrival
-      bar_sync_n(1, ncomp);
-      if (warp == 0 && lane == 0) mbar_arrive(&tl->afull[it & 1]);
-    }
-
-    // ---------------- phase B: row it-1
-    if (it > 0) {
-      const int p = it - 1;
-      const int pslot = p % kRing;
-      const int pk = k == 0 ? a.R - 1 : k - 1;
-      const int64_t punit = k == 0 ? unit - G : unit;
-      swait(&tl->rbar[pslot], (uint32_t)((p / kRing) & 1), tl, a.dev_err, kWsRow);
-      const Msg* rv = tl->recv[pslot];
-      const bool has = lane < (int)C;
-      const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
-                               has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, cT);
-      const bool gT_ok = !nm.badT && okT_p, gD_ok = !nm.badD && okD_p;
-      const float scT = gT_ok ? ex2((mwT_p - nm.MT) * cT) / nm.ST : 0.f;
-      const float scD = gD_ok ? ex2((mwD_p - nm.MD) * cT) / nm.SD : 0.f;
-      const bool bonus = pk == a.K;
-      const uint32_t tb = tcol + 64u * (uint32_t)(p & 1);
-      float eT[kEPT], eD[kEPT];
-      __syncwarp();  // the lanes left the wait above one by one
-#pragma unroll
-      for (int i = 0; i < kEPT; i += 8) {
-        tmem_ld8(tb + (uint32_t)i, &eT[i]);
-        tmem_ld8(tb + 32u + (uint32_t)i, &eD[i]);
-      }
-      tmem_wait_ld();
-      float tvw;
-      Cand cd = cand_empty();
-      if (scT > 0.f) {
-        // sum |p - q| = scT * sum |eT - eD * (scD / scT)|: one fused op per entry,
-        // exactly 0 for identical rows (ratio 1).
-        const float2 nr2 = f2(-(scD / scT));
-        float2 t2 = f2(0.f);
-#pragma unroll
-        for (int i = 0; i < kEPT; i += 2) {
-          const float2 d = __ffma2_rn(make_float2(eD[i], eD[i + 1]), nr2, make_float2(eT[i], eT[i + 1]));
-          t2 = __fadd2_rn(t2, make_float2(fabsf(d.x), fabsf(d.y)));
-        }
-        tvw = scT * (t2.x + t2.y);
-        if (bonus) {
-          // Tref = M/tau + g_min - margin bounds the winning score from below
-          const float margin = 1e-5f + 2e-7f * fabsf(nm.MT * a.inv_tau);
-          const float rho = ex2((mwT_p - nm.MT) * cT + (-kGumbelMinF + margin) * kLog2e);
-          const TIn* gT = (const TIn*)a.zT + (punit * a.R + pk) * a.ld + s0;
-          cd = bonus_screen<TIn>(tb, gT, s0, len, tid, ncomp, rho, a.inv_tau,
-                                 Stream(a.seed, a.round, SD_STREAM_BONUS), (uint32_t)punit);
-        }
-      } else {  // no target mass in this warp's entries (or a bad row): TV part = sum q
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < kEPT; ++i) s += eD[i];
-        tvw = scD * s;
-      }
-      tvw = warp_sum(tvw);
-      if (bonus) cd = warp_cand(cd);
-      if (lane == 0) {
-        tl->wtv[p & 1][warp] = tvw;
-        if (bonus) tl->wcand[p & 1][warp] = cd;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tl->bfull[p & 1]);
-    }
-
-    if (cur) {
-      mwT_p = mwTs;
-      mwD_p = mwDs;
-      okT_p = okT;
-      okD_p = okD;
-      if (++stage == nS) {
-        stage = 0;
-        phase ^= 1u;
-      }
-      if (++k == a.R) {
-        k = 0;
-        unit += G;
       }
     }
+    float sTw = accT.x + accT.y, sDw = accD.x + accD.y;
+    warp_sum2(sTw, sDw);
+    if (lane == 0) tl->wpart[it & 1][warp] = make_float4(mwT, sTw, mwD, sDw);
+    if (k == 0 && it > 0) screen(it - 1, unit - G);  // the previous row ended a particle
+    mwT_prev = mwT;
+    __syncwarp();
+    tmem_wait_st();
+    tmem_fence_before();
+    if (lane == 0) mbar_arrive(&tl->afull[it & 1]);
+    if (++stage == nS) {
+      stage = 0;
+      phase ^= 1u;
+    }
+    if (++k == a.R) {
+      k = 0;
+      unit += G;
+    }
+  }
+  if (nrows > 0) {  // the last row ends a particle too
+    screen(nrows - 1, unit - G);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tl->sfin);
   }
   __syncwarp();
   tmem_fence_before();
@@ -1860,9 +1899,9 @@ static bool make_plan(const void* fn, int V, int esize, int64_t units, LaunchPla
   return found;
 }
 
-// Launch plan of the pipelined SMC-SD kernel: one compute warp group per CTA
-// (32 entries per thread per row, at most 16 warps so that two TMEM row buffers
-// per warp fit) plus the communication and bookkeeping warps; the deepest ring
+// Launch plan of the SMC-SD kernel: producer warps covering the slice at 32
+// entries per thread per row (at most 16, so that two TMEM row buffers per
+// warp fit), four consumers and the two service warps; the deepest ring
 // that fits, and at least kMinSmem of shared memory so that one CTA runs per
 // SM (it takes all of the SM's tensor memory).  Among the cluster sizes it
 // keeps the most SMs busy for this many particles.
@@ -1886,8 +1925,8 @@ static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, Launc
   for (int C = 1; C <= kMaxCluster; ++C) {
     const int slice = (int)(((int64_t)(V + C - 1) / C + 7) / 8 * 8);
     const int ncomp = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
-    const int threads = ncomp + 64;  // + communication and bookkeeping warps
-    if (threads > kMaxThreads || ncomp / 32 > kMaxWarps) continue;
+    const int threads = ncomp + 32 * (kConsumers + 2);  // + consumers, communication, bookkeeping
+    if (threads > kMaxThreadsSmc || ncomp / 32 > kMaxWarps) continue;
     const uint32_t sb = (uint32_t)(((int64_t)slice * esize + 127) / 128 * 128);
     int nS = 0;
     for (int st = kMaxStages; st >= 2; --st)
@@ -1996,6 +2035,7 @@ static void fill_common(ScoreArgs& a, float tau) {
   a.inv_tau = (float)(1.0 / (double)tau);
   a.cT = (float)(1.4426950408889634 / (double)tau);
   a.tau64 = (double)tau;
+  a.inv_tau64 = 1.0 / (double)tau;
 }
 
 }  // namespace smcsd

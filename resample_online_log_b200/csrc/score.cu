@@ -1069,6 +1069,7 @@ struct alignas(16) BMsg {  // one slice's phase-B results for the leader
 
 struct alignas(128) SmcTail {
   uint64_t full[kMaxStages];    // ring stages (target and draft slices of one row)
+  uint64_t empty[kMaxStages];   // producers done reading a stage
   uint64_t afull[2];  // producers done with a row (exps in TMEM, partials posted)
   uint64_t bfull[2];  // consumers done with a row (TV partials, candidates posted)
   uint64_t tfree[2];  // consumers done reading a TMEM row buffer
@@ -1284,39 +1285,42 @@ __device__ __forceinline__ uint4 load_chunk(const TIn* st, const TIn* g, int e0,
 }
 
 // Bonus-token screen over this thread's target entries of a particle's last
-// row, from the exps held in TMEM (relative to the warp max): entries whose
-// y = e * rho = e^{a - Tref} proves they cannot win are dropped before any
-// log, groups of four far below Tref before the Philox call; the few kept
-// entries re-read their logit from HBM and become candidates with fp32
-// bounds.  Its loop stays rolled: one row in K+1 needs it.
+// row, from the exps held in TMEM (relative to the warp max): the Philox words
+// are drawn four blocks at a time (independent, so they overlap); an
+// entry whose y = e * rho = e^{a - Tref} proves it cannot win is dropped
+// before any log; the few kept entries re-read their logit from HBM and
+// become candidates with fp32 bounds.
 template <typename TIn>
 __device__ __forceinline__ Cand bonus_screen(uint32_t tcolT, const TIn* g, int s0, int len, int tid,
                                              int ncomp, float rho, float inv_tau, const Stream bst,
                                              uint32_t rowid) {
   constexpr int EPC = Chunk<TIn>::EPC;
+  float e[kEPT];
+  __syncwarp();
+  tmem_ld32(tcolT, e);
+  tmem_wait_ld();
   Cand cd = cand_empty();
-#pragma unroll 1
-  for (int i8 = 0; i8 < kEPT; i8 += 8) {
-    float e[8];
-    __syncwarp();  // converge after the divergent screening of the previous block
-    tmem_ld8(tcolT + (uint32_t)i8, e);
-    tmem_wait_ld();
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int i = i8 + 4 * q;  // this thread's entry index: chunk i / EPC, offset i % EPC
+  for (int h = 0; h < 2; ++h) {  // two halves of four independent Philox blocks each
+    U4 w[kEPT / 8];
+#pragma unroll
+    for (int q = 0; q < kEPT / 8; ++q) {  // entries i..i+3 of this thread: one Philox block
+      const int i = 16 * h + 4 * q;
       const int eg = (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
-      float y[4];
+      w[q] = bst.at((uint32_t)((s0 + eg) >> 2), rowid);
+    }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) y[j] = e[4 * q + j] * rho;
-      if (eg >= len || fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3])) < kYSkip) continue;
-      const int v0 = s0 + eg;
-      const U4 w = bst.at((uint32_t)(v0 >> 2), rowid);
-      const float u[4] = {uniform_f32(w.x), uniform_f32(w.y), uniform_f32(w.z), uniform_f32(w.w)};
+    for (int q = 0; q < kEPT / 8; ++q) {
+      const int i = 16 * h + 4 * q;
+      const int eg = (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (!keep_bonus(y[j], u[j]) || eg + j >= len) continue;
-        const float z = Elem<TIn>::get(g, eg + j);
-        if (z > -INFINITY) cd = cand_merge(cd, bonus_cand_z(z, u[j], inv_tau, v0 + j));
+        const float y = e[i + j] * rho;
+        const float u = uniform_f32(word_of(w[q], j));
+        if (keep_bonus(y, u) && eg + j < len) {
+          const float z = Elem<TIn>::get(g, eg + j);
+          if (z > -INFINITY) cd = cand_merge(cd, bonus_cand_z(z, u, inv_tau, s0 + eg + j));
+        }
       }
     }
   }
@@ -1482,7 +1486,10 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
   const float cT = a.cT;
 
   if (tid == 0) {
-    for (int st = 0; st < nS; ++st) mbar_init(&tl->full[st], 1);
+    for (int st = 0; st < nS; ++st) {
+      mbar_init(&tl->full[st], 1);
+      mbar_init(&tl->empty[st], (uint32_t)nA);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tl->afull[b], (uint32_t)nA);
       mbar_init(&tl->bfull[b], kConsumers);
@@ -1528,9 +1535,12 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       for (int i = 0; i < nS && i < nrows; ++i) issue(i, i);
     int k = 0, stage = 0;  // position and ring stage of row it
     for (int it = 0; it <= nrows; ++it) {
-      if (it < nrows) {  // row it: the producers are done with it and with its stage
+      if (it < nrows) {  // row it: refill its stage once read, then its message
+        if (it + nS < nrows) {
+          swait(&tl->empty[stage], (uint32_t)((it / nS) & 1), tl, a.dev_err, kWsAfull);
+          if (lane == 0) issue(it + nS, stage);
+        }
         swait(&tl->afull[it & 1], (uint32_t)((it >> 1) & 1), tl, a.dev_err, kWsAfull);
-        if (lane == 0 && it + nS < nrows) issue(it + nS, stage);
         const float4 wp =
             lane < nA ? tl->wpart[it & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
         float mT = wp.x, mD = wp.z;
@@ -1616,32 +1626,26 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
           // sum |p - q| = scT * sum |eT - eD * (scD / scT)|: one fused op per entry,
           // exactly 0 for identical rows (ratio 1).
           const float2 nr2 = f2(-(scD / scT));
-          float2 t2 = f2(0.f);
+          float eT[kEPT], eD[kEPT];
+          tmem_ld32(tb, eT);
+          tmem_ld32(tb + 32u, eD);
+          tmem_wait_ld();
+          float2 t2 = f2(0.f), u2 = f2(0.f);
 #pragma unroll
-          for (int i = 0; i < kEPT; i += 16) {
-            float eT[16], eD[16];
-            tmem_ld8(tb + (uint32_t)i, &eT[0]);
-            tmem_ld8(tb + (uint32_t)i + 8u, &eT[8]);
-            tmem_ld8(tb + 32u + (uint32_t)i, &eD[0]);
-            tmem_ld8(tb + 40u + (uint32_t)i, &eD[8]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; j += 2) {
-              const float2 d = __ffma2_rn(make_float2(eD[j], eD[j + 1]), nr2, make_float2(eT[j], eT[j + 1]));
-              t2 = __fadd2_rn(t2, make_float2(fabsf(d.x), fabsf(d.y)));
-            }
+          for (int j = 0; j < kEPT; j += 4) {
+            const float2 d0 = __ffma2_rn(make_float2(eD[j], eD[j + 1]), nr2, make_float2(eT[j], eT[j + 1]));
+            const float2 d1 = __ffma2_rn(make_float2(eD[j + 2], eD[j + 3]), nr2, make_float2(eT[j + 2], eT[j + 3]));
+            t2 = __fadd2_rn(t2, make_float2(fabsf(d0.x), fabsf(d0.y)));
+            u2 = __fadd2_rn(u2, make_float2(fabsf(d1.x), fabsf(d1.y)));
           }
-          tv += scT * (t2.x + t2.y);
+          tv += scT * ((t2.x + t2.y) + (u2.x + u2.y));
         } else if (scD > 0.f) {  // no target mass in these entries (or a bad row): TV part = sum q
+          float eD[kEPT];
+          tmem_ld32(tb + 32u, eD);
+          tmem_wait_ld();
           float sq = 0.f;
 #pragma unroll
-          for (int i = 0; i < kEPT; i += 8) {
-            float eD[8];
-            tmem_ld8(tb + 32u + (uint32_t)i, eD);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 8; ++j) sq += eD[j];
-          }
+          for (int j = 0; j < kEPT; ++j) sq += eD[j];
           tv += scD * sq;
         }
       }
@@ -1730,6 +1734,10 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
         tl->zx[it & 1][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
       }
     }
+    if (HOLD) {  // the stage is in registers now: it can be refilled
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->empty[stage]);
+    }
     float mwT = CK::acc_f32(aT), mwD = CK::acc_f32(aD);
     warp_max2_nan(mwT, mwD);
     const float mwTs = mwT == -INFINITY ? 0.f : mwT;
@@ -1772,6 +1780,10 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
           tmem_st8(tb + 32u + col, eD);
         }
       }
+    }
+    if (!HOLD) {  // pass 2 re-read the stage
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->empty[stage]);
     }
     float sTw = accT.x + accT.y, sDw = accD.x + accD.y;
     warp_sum2(sTw, sDw);

@@ -11,6 +11,7 @@ scaling, no collective on the data path; barrier + max-over-ranks timing).
 """
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -27,6 +28,38 @@ import torch  # noqa: E402
 
 METRIC = "verify+resample logit rows/s; achieved HBM TB/s as fraction of B200 peak"
 WORKLOAD = "smc_scale"
+
+
+KERNEL_SOURCES = ["resample_online_log_b200/csrc/score.cu", "resample_online_log_b200/csrc/common.cuh"]
+TRAFFIC_SUMMARY = "profiles/smc_kernel_smc_scale.md"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(B):
+    """DRAM bytes (read + write) of one score-kernel launch over B sequences, from
+    the committed ncu summary, if it was taken on the current kernel sources."""
+    path = os.path.join(ROOT, TRAFFIC_SUMMARY)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("- ") and ":" in line:
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    try:
+        if fields.get("source_sha256") != kernel_source_hash():
+            return None
+        return float(fields["dram_bytes_per_sequence"]) * B
+    except (KeyError, ValueError):
+        return None
 
 
 def peaks():
@@ -264,10 +297,10 @@ def run_ours(args, rank, world, local):
         "config": {"workload": WORKLOAD if not args.sequences else f"{WORKLOAD}[B={B}]",
                    "B": B, "N": N, "K": K, "V": V, "logits": cfg.dtype,
                    "tau": cfg.tau, "pages_per_particle": P, "parallelism": f"replicas{world}",
-                   "l2": "inputs (37.8 GB) larger than L2; no flush"},
+                   "l2": f"inputs ({2 * rows_per_step * V * esize / 1e9:.1f} GB) larger than L2; no flush"},
         "hbm_TBps_score": achieved / 1e3,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "score_kernel",
+                     "frac": achieved / hbm_peak, "traffic": measured_traffic(B), "kernel": "smc_kernel",
                      "peak_kind": peak_kind, "score_ms": score_ms,
                      "algorithmic_bytes": alg_bytes},
         "gpu_launches": 3 * args.steps,

@@ -1201,9 +1201,8 @@ __device__ __noinline__ int exact_bonus_row(const TIn* row, int V, double tau64,
 
 // Candidate from one kept entry: a = z / tau in fp32, Gumbel in fp32, with
 // bounds that contain the exact fp64 score.
-__device__ __noinline__ Cand bonus_cand_z(float z, float u, float inv_tau, int v) {
+__device__ __noinline__ Cand bonus_cand_a(float a32, float u, int v) {
   const float g32 = gumbel_f32(u);
-  const float a32 = z * inv_tau;
   Cand cd;
   cd.s = a32 + g32;
   const float d = 4e-6f + 4.8e-7f * (fabsf(a32) + 2.f * fabsf(g32));
@@ -1288,11 +1287,12 @@ __device__ __forceinline__ uint4 load_chunk(const TIn* st, const TIn* g, int e0,
 // row, from the exps held in TMEM (relative to the warp max): the Philox words
 // are drawn four blocks at a time (independent, so they overlap); an
 // entry whose y = e * rho = e^{a - Tref} proves it cannot win is dropped
-// before any log; the few kept entries re-read their logit from HBM and
-// become candidates with fp32 bounds.
+// before any log; the few kept entries become candidates with fp32 bounds,
+// their logit over tau recovered as a = m/tau + ln(e) (m: the warp max the exp
+// is relative to; the error is far inside the candidate bounds).
 template <typename TIn>
-__device__ __forceinline__ Cand bonus_screen(uint32_t tcolT, const TIn* g, int s0, int len, int tid,
-                                             int ncomp, float rho, float inv_tau, const Stream bst,
+__device__ __forceinline__ Cand bonus_screen(uint32_t tcolT, int s0, int len, int tid, int ncomp,
+                                             float rho, float mw_a, const Stream bst,
                                              uint32_t rowid) {
   constexpr int EPC = Chunk<TIn>::EPC;
   float e[kEPT];
@@ -1317,10 +1317,8 @@ __device__ __forceinline__ Cand bonus_screen(uint32_t tcolT, const TIn* g, int s
       for (int j = 0; j < 4; ++j) {
         const float y = e[i + j] * rho;
         const float u = uniform_f32(word_of(w[q], j));
-        if (keep_bonus(y, u) && eg + j < len) {
-          const float z = Elem<TIn>::get(g, eg + j);
-          if (z > -INFINITY) cd = cand_merge(cd, bonus_cand_z(z, u, inv_tau, s0 + eg + j));
-        }
+        if (keep_bonus(y, u) && eg + j < len && e[i + j] > 0.f)
+          cd = cand_merge(cd, bonus_cand_a(mw_a + logf(e[i + j]), u, s0 + eg + j));
       }
     }
   }
@@ -1617,10 +1615,11 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
                                has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, cT);
       float tv = 0.f;
+      const float invST = 1.f / nm.ST, invSD = 1.f / nm.SD;
       for (int w = q; w < nA; w += 4) {
         const float4 wp = tl->wpart[p & 1][w];  // producer w's raw maxima and sums
-        const float scT = (!nm.badT && wp.x > -INFINITY) ? ex2((wp.x - nm.MT) * cT) / nm.ST : 0.f;
-        const float scD = (!nm.badD && wp.z > -INFINITY) ? ex2((wp.z - nm.MD) * cT) / nm.SD : 0.f;
+        const float scT = (!nm.badT && wp.x > -INFINITY) ? ex2((wp.x - nm.MT) * cT) * invST : 0.f;
+        const float scD = (!nm.badD && wp.z > -INFINITY) ? ex2((wp.z - nm.MD) * cT) * invSD : 0.f;
         const uint32_t tb = tq + 128u * (uint32_t)(w >> 2) + 64u * (uint32_t)(p & 1);
         if (scT > 0.f) {
           // sum |p - q| = scT * sum |eT - eD * (scD / scT)|: one fused op per entry,
@@ -1687,9 +1686,9 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       // Tref = M/tau + g_min - margin bounds the winning score from below
       const float margin = 1e-5f + 2e-7f * fabsf(nm.MT * a.inv_tau);
       const float rho = ex2((mwT_prev - nm.MT) * cT + (-kGumbelMinF + margin) * kLog2e);
-      const TIn* gT = (const TIn*)a.zT + (punit * a.R + a.K) * a.ld + s0;
-      cd = bonus_screen<TIn>(tcol + 64u * (uint32_t)(p & 1), gT, s0, len, tid, ncomp, rho,
-                             a.inv_tau, Stream(a.seed, a.round, SD_STREAM_BONUS), (uint32_t)punit);
+      cd = bonus_screen<TIn>(tcol + 64u * (uint32_t)(p & 1), s0, len, tid, ncomp, rho,
+                             mwT_prev * a.inv_tau, Stream(a.seed, a.round, SD_STREAM_BONUS),
+                             (uint32_t)punit);
     }
     cd = warp_cand(cd);
     if (lane == 0) tl->wcand[p & 3][warp] = cd;

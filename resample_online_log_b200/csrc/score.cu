@@ -1082,7 +1082,12 @@ struct alignas(128) SmcTail {
   float4 wpart[2][kMaxWarps];
   float wtv[2][kConsumers];
   Cand wcand[4][kMaxWarps];  // producers' bonus candidates, by row & 3
-  float zx[2][2];
+  // Raw logits of a row's draft token at its owner, by row & 3: producer warps
+  // are not ordered among themselves, so the owner may post row it+2's value
+  // before the slowest warp has finished row it (and so before the
+  // communication warp has read it); row it+3 needs row it's TMEM buffer back,
+  // which comes after that read.
+  float zx[4][2];
 };
 
 // Wait sites, reported in bits 8..15 of the error word with SD_DEV_TIMEOUT.
@@ -1232,6 +1237,9 @@ struct Chunk<uint16_t> {
     const uint32_t w = (j >> 1) == 0 ? v.x : ((j >> 1) == 1 ? v.y : ((j >> 1) == 2 ? v.z : v.w));
     return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
   }
+  static __device__ __forceinline__ uint4 neg_inf() {
+    return make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+  }
   static __device__ __noinline__ uint4 gather(const uint16_t* st, const uint16_t* g, int e0, int len,
                                               int tma_len) {
     uint32_t w[4];
@@ -1261,6 +1269,9 @@ struct Chunk<float> {
   static __device__ __forceinline__ float elem(const uint4& v, int j) {  // j: compile-time
     return __uint_as_float(j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w)));
   }
+  static __device__ __forceinline__ uint4 neg_inf() {
+    return make_uint4(0xFF800000u, 0xFF800000u, 0xFF800000u, 0xFF800000u);
+  }
   static __device__ __noinline__ uint4 gather(const float* st, const float* g, int e0, int len,
                                               int tma_len) {
     uint32_t w[4];
@@ -1275,11 +1286,13 @@ struct Chunk<float> {
 };
 
 // Chunk starting at slice entry e0: from the ring stage where the bulk copy
-// covered it, else from HBM; entries past the slice read as -inf.
+// covered it, else from HBM; entries past the slice read as -inf (a chunk
+// wholly past it without a call: the last lanes of a CTA hold such chunks).
 template <typename TIn>
 __device__ __forceinline__ uint4 load_chunk(const TIn* st, const TIn* g, int e0, int len,
                                             int tma_len) {
   if (e0 + Chunk<TIn>::EPC <= tma_len) return *reinterpret_cast<const uint4*>(st + e0);
+  if (e0 >= len) return Chunk<TIn>::neg_inf();
   return Chunk<TIn>::gather(st, g, e0, len, tma_len);
 }
 
@@ -1547,8 +1560,8 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
         warp_sum2(sumT, sumD);
         float zxT = 0.f, zxD = 0.f;
         if (k < a.K) {
-          zxT = tl->zx[it & 1][0];
-          zxD = tl->zx[it & 1][1];
+          zxT = tl->zx[it & 3][0];
+          zxD = tl->zx[it & 3][1];
         }
         const int slot = it % kRing;
         // Once this message is out, the other CTAs can send rows up to it + kLead;
@@ -1729,8 +1742,8 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
     if (x >= s0 && x < s0 + len) {  // the owner of the draft token records its raw logits
       const int le = x - s0;
       if (((le / EPC) % ncomp) == tid) {
-        tl->zx[it & 1][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
-        tl->zx[it & 1][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
+        tl->zx[it & 3][0] = le < tma_len ? Elem<TIn>::get(stT, le) : Elem<TIn>::get(gT, le);
+        tl->zx[it & 3][1] = le < tma_len ? Elem<TIn>::get(stD, le) : Elem<TIn>::get(gD, le);
       }
     }
     if (HOLD) {  // the stage is in registers now: it can be refilled

@@ -174,6 +174,34 @@ def test_reruns_bit_identical():
         assert np.array_equal(a[key], b[key], equal_nan=True), key
 
 
+def check_all_rows(d, cfg, logw, tv, lp, lse, name):
+    """Identities every row of a whole config must satisfy, checked on the device
+    for all particles (the oracle comparison above covers sampled sequences):
+    lp + lse equals the draft token's logit over tau (a gather of the input);
+    logw is the sum over k of lp - lq; max_v z/tau <= lse <= max_v z/tau + log V;
+    0 <= tv <= 1."""
+    B, N, R, V, K = cfg.B, cfg.N, cfg.R, cfg.V, cfg.K
+    U = B * N
+    zT, zD = d["zT"].view(U, R, -1), d["zD"].view(U, R, -1)
+    lp, lse = lp.view(U, K, 2), lse.view(U, R, 2)
+    x = d["draft"].view(U, K, 1).long()
+    tau = float(np.float32(cfg.tau))  # the C ABI takes tau in fp32
+    for h, z in enumerate((zT, zD)):
+        zx = z[:, :K].gather(2, x).squeeze(2).double() / tau
+        got = lp[..., h] + lse[:, :K, h]
+        bad = (got - zx).abs() > 1e-9 * (1.0 + zx.abs())
+        assert not bad.any(), f"{name}: lp + lse != z[x]/tau at (unit, k) {bad.nonzero()[:8].tolist()}"
+        mx = torch.cat([z[u0:u0 + 512].amax(2) for u0 in range(0, U, 512)]).double() / tau
+        # (the slice sums are fp32, so the lower bound holds to their rounding)
+        lo_ok = lse[..., h] >= mx - 1e-6 * (1.0 + mx.abs())
+        hi_ok = lse[..., h] <= mx + float(np.log(V)) + 1e-6 * (1.0 + mx.abs())
+        assert bool((lo_ok & hi_ok).all()), f"{name}: lse outside [max, max + log V]"
+    s = (lp[..., 0] - lp[..., 1]).sum(1)
+    lw = logw.view(U)
+    assert bool(((lw - s).abs() <= 1e-9 * (1.0 + s.abs())).all()), f"{name}: logw != sum(lp - lq)"
+    assert bool(((tv >= 0) & (tv <= 1 + 1e-6)).all()), f"{name}: tv outside [0, 1]"
+
+
 @pytest.mark.parametrize("name,seqs", [("smc_batch", [0, 37]), ("smc_scale", [5, 200])])
 def test_full_size_config_sampled(name, seqs):
     """Whole config on the GPU (inputs built on the device), sampled sequences checked
@@ -187,11 +215,13 @@ def test_full_size_config_sampled(name, seqs):
     out_bonus = torch.empty((B, N), dtype=torch.int32, device="cuda")
     out_tv = torch.empty((B, N, R), dtype=torch.float32, device="cuda")
     out_lp = torch.empty((B, N, K, 2), dtype=torch.float64, device="cuda")
+    out_lse = torch.empty((B, N, R, 2), dtype=torch.float64, device="cuda")
     err = torch.zeros((1,), dtype=torch.int32, device="cuda")
     lib.smcsd_score(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed, 1, out_logw, out_bonus,
-                    tv_out=out_tv, lp_out=out_lp, dev_err=err)
+                    tv_out=out_tv, lp_out=out_lp, lse_out=out_lse, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
+    check_all_rows(d, cfg, out_logw, out_tv, out_lp, out_lse, name)
     for b in seqs:
         h = gen.gen_config_rows(cfg, seqs=[b])
         dev_t = d["zT"][b].float().cpu().numpy()

@@ -1111,23 +1111,15 @@ __device__ __forceinline__ void swait(uint64_t* bar, uint32_t parity, SmcTail* t
 }
 
 // Paired warp reductions (two independent values per shuffle round).
+// Warp maxima in one instruction each (redux.sync on f32, sm_100a): NaN inputs
+// are dropped (as fmaxf does), or with .NaN make the result NaN.
 __device__ __forceinline__ void warp_max2(float& a, float& b) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float x = __shfl_xor_sync(0xffffffffu, a, o);
-    const float y = __shfl_xor_sync(0xffffffffu, b, o);
-    a = fmaxf(a, x);
-    b = fmaxf(b, y);
-  }
+  asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(a));
+  asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(b));
 }
 __device__ __forceinline__ void warp_max2_nan(float& a, float& b) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float x = __shfl_xor_sync(0xffffffffu, a, o);
-    const float y = __shfl_xor_sync(0xffffffffu, b, o);
-    a = fmax_nan(a, x);
-    b = fmax_nan(b, y);
-  }
+  asm volatile("redux.sync.max.NaN.f32 %0, %0, 0xffffffff;" : "+f"(a));
+  asm volatile("redux.sync.max.NaN.f32 %0, %0, 0xffffffff;" : "+f"(b));
 }
 __device__ __forceinline__ void warp_sum2(float& a, float& b) {
 #pragma unroll

@@ -1289,41 +1289,52 @@ __device__ __forceinline__ uint4 load_chunk(const TIn* st, const TIn* g, int e0,
 }
 
 // Bonus-token screen over this thread's target entries of a particle's last
-// row, from the exps held in TMEM (relative to the warp max): the Philox words
-// are drawn four blocks at a time (independent, so they overlap); an
-// entry whose y = e * rho = e^{a - Tref} proves it cannot win is dropped
-// before any log; the few kept entries become candidates with fp32 bounds,
-// their logit over tau recovered as a = m/tau + ln(e) (m: the warp max the exp
-// is relative to; the error is far inside the candidate bounds).
+// row, from the exps held in TMEM (relative to the warp max), in two halves of
+// sixteen entries (one loop body, kept small for the instruction cache): the
+// four Philox blocks of a half are drawn together (independent, so they
+// overlap); an entry whose y = e * rho = e^{a - Tref} proves it cannot win is
+// dropped before any log; the few kept entries become candidates with fp32
+// bounds, their logit over tau recovered as a = m/tau + ln(e) (m: the warp max
+// the exp is relative to; the error is far inside the candidate bounds).
 template <typename TIn>
 __device__ __forceinline__ Cand bonus_screen(uint32_t tcolT, int s0, int len, int tid, int ncomp,
                                              float rho, float mw_a, const Stream bst,
                                              uint32_t rowid) {
   constexpr int EPC = Chunk<TIn>::EPC;
-  float e[kEPT];
-  __syncwarp();
-  tmem_ld32(tcolT, e);
-  tmem_wait_ld();
   Cand cd = cand_empty();
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    float e[16];
+    __syncwarp();
+    tmem_ld16(tcolT + 16u * (uint32_t)h, e);
+    tmem_wait_ld();
+    // One bound for the half: with y <= ymax = emax * rho, keep_bonus needs
+    // u >= thr(ymax) (same fp32 steps, monotone), so a word whose top 23 bits
+    // m = w >> 9 fall below mstar fails for every entry here;
+    // u = (m + 1/2) 2^-23 >= thr  <=>  m >= thr 2^23 - 1/2 (exact in fp32).
+    float emax = 0.f;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {  // two halves of four independent Philox blocks each
-    U4 w[kEPT / 8];
+    for (int i = 0; i < 16; ++i) emax = fmaxf(emax, e[i]);
+    const float thr = (1.0f - (emax * rho) * 1.001f) - 2.4e-7f;
+    const uint32_t mstar = thr > 0.f ? (uint32_t)ceilf(thr * 8388608.f - 0.5f) : 0u;
+    U4 w[4];
 #pragma unroll
-    for (int q = 0; q < kEPT / 8; ++q) {  // entries i..i+3 of this thread: one Philox block
+    for (int q = 0; q < 4; ++q) {  // entries 16h + 4q .. +3 of this thread: one Philox block
       const int i = 16 * h + 4 * q;
       const int eg = (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
       w[q] = bst.at((uint32_t)((s0 + eg) >> 2), rowid);
     }
 #pragma unroll
-    for (int q = 0; q < kEPT / 8; ++q) {
+    for (int q = 0; q < 4; ++q) {
       const int i = 16 * h + 4 * q;
       const int eg = (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float y = e[i + j] * rho;
+        if ((word_of(w[q], j) >> 9) < mstar) continue;
+        const float ej = e[4 * q + j];
         const float u = uniform_f32(word_of(w[q], j));
-        if (keep_bonus(y, u) && eg + j < len && e[i + j] > 0.f)
-          cd = cand_merge(cd, bonus_cand_a(mw_a + logf(e[i + j]), u, s0 + eg + j));
+        if (keep_bonus(ej * rho, u) && eg + j < len && ej > 0.f)
+          cd = cand_merge(cd, bonus_cand_a(mw_a + logf(ej), u, s0 + eg + j));
       }
     }
   }

@@ -1393,8 +1393,6 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
           zxD = o.zxD;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tl->adone[slot]);  // this row's message slot is read
       if (lane == 0) {
         if (bad_cur) raise_err(a.dev_err, SD_DEV_NONFINITE);
         if (a.lse_out) {
@@ -1437,17 +1435,22 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
       const BMsg* bm = tl->brecv[pslot];
       const bool has = lane < (int)C;
       float tv = has ? bm[lane].tv : 0.f;
+      Cand c = cand_empty();
+      if (pk == a.K && has) {
+        c.s = bm[lane].s;
+        c.lo = bm[lane].lo;
+        c.hi = bm[lane].hi;
+        c.ohi = bm[lane].ohi;
+        c.idx = bm[lane].idx;
+      }
+      // Both of row p's slots (row message and leader message) are read: the
+      // CTAs may now run far enough ahead to refill them (the leader's
+      // communication warp waits for this before each row message).
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->adone[pslot]);
       tv = warp_sum(tv);
       if (want_tv && lane == 0) a.tv_out[punit * a.R + pk] = prev_bad ? NAN : 0.5f * tv;
       if (pk == a.K) {
-        Cand c = cand_empty();
-        if (has) {
-          c.s = bm[lane].s;
-          c.lo = bm[lane].lo;
-          c.hi = bm[lane].hi;
-          c.ohi = bm[lane].ohi;
-          c.idx = bm[lane].idx;
-        }
         c = warp_cand(c);
         int winner;
         if (prev_badT || c.idx == 0x7FFFFFFF) winner = -1;

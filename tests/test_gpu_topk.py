@@ -64,6 +64,28 @@ def test_dense_peaked_and_masked_rows():
     assert list(g["idx"][1, 3:]) == [-1] * 5
 
 
+def check_all_rows(z, cfg, idx, sc, lp):
+    """Identities every row of the whole config must satisfy (the oracle covers
+    sampled rows): indices in range and distinct; logp = z[idx]/tau - lse (a
+    gather of the input and the row's log-sum-exp, fp64); score - z[idx]/tau is a
+    Gumbel of a 23-bit uniform, so it lies in [g_min, g_max]; scores are
+    non-increasing along k."""
+    rows, V = z.shape
+    tau = float(np.float32(cfg.tau))  # the C ABI takes tau in fp32
+    assert bool(((idx >= 0) & (idx < V)).all()), "topk: index out of range"
+    srt = idx.sort(dim=1).values
+    assert bool((srt[:, 1:] != srt[:, :-1]).all()), "topk: repeated index in a row"
+    lse = torch.cat([torch.logsumexp(z[r0:r0 + 256].double() / tau, dim=1)
+                     for r0 in range(0, rows, 256)])
+    a = z.gather(1, idx.long()).double() / tau
+    dl = (lp.double() - (a - lse[:, None])).abs()
+    assert bool((dl <= 1e-5 * (1.0 + a.abs())).all()), f"topk: logp off by {float(dl.max()):.3e}"
+    g = sc.double() - a
+    g_min, g_max = -2.8104282144774236, 16.635532333438686
+    assert bool(((g >= g_min - 1e-4) & (g <= g_max + 1e-4)).all()), "topk: score - z/tau not a Gumbel"
+    assert bool((sc[:, 1:] <= sc[:, :-1]).all()), "topk: scores not in descending order"
+
+
 def test_dense_config_sampled():
     """Whole 4096 x 152064 config on the device; sampled rows against the oracle on
     host-built rows (same bytes)."""
@@ -79,6 +101,7 @@ def test_dense_config_sampled():
     lib.gumbel_topk(z, cfg.topk, cfg.tau, cfg.seed, 2, idx, score_out=sc, logp_out=lp, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
+    check_all_rows(z, cfg, idx, sc, lp)
     for r in [0, 1, 2047, 4095]:
         h = gen.gen_config_rows(cfg, seqs=[r])
         assert np.array_equal(z[r].float().cpu().numpy(), h["z"][0])

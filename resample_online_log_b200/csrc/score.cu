@@ -1058,6 +1058,7 @@ constexpr int kMaxStages = 4;
 constexpr uint32_t kTmemCols = 512;  // all of the SM's tensor memory (one CTA per SM)
 constexpr int kConsumers = 4;        // phase-B warps, one per TMEM lane quarter
 constexpr int kMaxThreadsSmc = 640;  // up to 14 producers + 4 consumers + 2 service warps
+static_assert(kMaxThreadsSmc / 32 - kConsumers - 2 <= 16, "one lane per producer in each half-warp");
 constexpr size_t kMinSmem = 120 * 1024;  // > half an SM's shared memory: one CTA per SM
 
 struct alignas(16) BMsg {  // one slice's phase-B results for the leader
@@ -1633,17 +1634,30 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       const bool has = lane < (int)C;
       const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
                                has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, cT);
+      // Scale factors of all producers at once (one exp2 and one division per
+      // lane instead of a chain per producer): lane w < 16 takes producer w's
+      // target half, lane 16 + w its draft half; lanes < 16 also -scD / scT.
+      const int wl = lane & 15;
+      const bool hD = lane >= 16;
+      const float4 wq =
+          wl < nA ? tl->wpart[p & 1][wl] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+      const float mwl = hD ? wq.z : wq.x;
+      const bool badl = hD ? nm.badD : nm.badT;
+      const float scl = (!badl && mwl > -INFINITY)
+                            ? ex2((mwl - (hD ? nm.MD : nm.MT)) * cT) * (1.f / (hD ? nm.SD : nm.ST))
+                            : 0.f;
+      const float sco = __shfl_xor_sync(0xffffffffu, scl, 16);
+      const float nrl = scl > 0.f ? -(sco / scl) : 0.f;
       float tv = 0.f;
-      const float invST = 1.f / nm.ST, invSD = 1.f / nm.SD;
       for (int w = q; w < nA; w += 4) {
-        const float4 wp = tl->wpart[p & 1][w];  // producer w's raw maxima and sums
-        const float scT = (!nm.badT && wp.x > -INFINITY) ? ex2((wp.x - nm.MT) * cT) * invST : 0.f;
-        const float scD = (!nm.badD && wp.z > -INFINITY) ? ex2((wp.z - nm.MD) * cT) * invSD : 0.f;
+        const float scT = __shfl_sync(0xffffffffu, scl, w);
+        const float scD = __shfl_sync(0xffffffffu, scl, w + 16);
+        const float nr = __shfl_sync(0xffffffffu, nrl, w);
         const uint32_t tb = tq + 128u * (uint32_t)(w >> 2) + 64u * (uint32_t)(p & 1);
         if (scT > 0.f) {
           // sum |p - q| = scT * sum |eT - eD * (scD / scT)|: one fused op per entry,
           // exactly 0 for identical rows (ratio 1).
-          const float2 nr2 = f2(-(scD / scT));
+          const float2 nr2 = f2(nr);
           float eT[kEPT], eD[kEPT];
           tmem_ld32(tb, eT);
           tmem_ld32(tb + 32u, eD);

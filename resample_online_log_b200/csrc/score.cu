@@ -1104,7 +1104,7 @@ __device__ __forceinline__ void swait(uint64_t* bar, uint32_t parity, SmcTail* t
   if (mbar_try_wait(bar, parity)) return;
   volatile int* ab = &tl->abort_flag;
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (*ab) return;
+    if ((i & 15u) == 0 && *ab) return;  // (a shared-memory read every 16 polls only)
     if (mbar_try_wait(bar, parity)) return;
   }
   *ab = 1;

@@ -14,6 +14,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -35,11 +36,19 @@ NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (the measured copy peak is the d
 TRAFFIC_SUMMARY = "profiles/smc_kernel_smc_scale.md"
 
 
+def _code_only(text):
+    """Source text without comments and with whitespace runs collapsed, so that a
+    comment-only edit keeps the hash (the compiled kernel is the same)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1037,11 +1037,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) score_kernel(const ScoreArgs a
 //   producers (one per 32 x 32 entries of the slice), row by row: move the
 //     row's slices from the ring to registers, warp maxima, exps (one MUFU
 //     exp2 per entry) and sums; the exps of both halves go to tensor memory
-//     (TMEM, two row buffers per warp); post the (max, sum) partials.
+//     (TMEM, two row buffers per warp); post the (max, sum) partials.  In the
+//     row after a particle's last row they also screen that row's bonus-token
+//     candidates from its exps, still in TMEM.
 //   consumers (four, one per TMEM lane quarter), one row behind: once the
 //     row's messages are in, rebuild its normalisers, read the exps back from
-//     TMEM and take the TV partial sum |p - q|; on a particle's last row also
-//     screen the bonus-token candidates; then hand the row buffer back.
+//     TMEM and take the TV partial sum |p - q|; then hand the row buffer back.
 //   communication: turns the producers' partials into one 32-byte message per
 //     row for every CTA of the cluster (st.async into distributed shared
 //     memory, completing on the receiver's mbarrier -- no cluster barrier on

@@ -358,6 +358,107 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def run_rows(args, workload):
+    """The other rows of the path, each on its own configuration (one GPU, one
+    JSON line each): `verify` = standard SD verification of 128 sequences x
+    (5+1) target / 5 draft rows of V = 32000 bf16 (90 MB, below L2: L2 flushed
+    before every launch); `topk` = Gumbel-top-8 over 4096 x 152064 bf16 rows
+    (1.25 GB) and the sparse variant over 4096 x top-10 stored rows.  Each line
+    has the kernel's event-timed mean, its algorithmic bytes against the
+    measured copy bandwidth, and the oracle timed on a sample of the same rows."""
+    import oracle
+    import resample_online_log_b200 as lib
+    from synth import device as sdev
+    from synth import gen
+
+    cfg = gen.CONFIGS[workload]
+    dev = "cuda"
+    hbm_peak, peak_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2x L2
+    err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(call, flush_l2):
+        for i in range(args.warmup):
+            call(i)
+        torch.cuda.synchronize()
+        ts = []
+        for i in range(args.steps):
+            if flush_l2:
+                flush.add_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call(args.warmup + i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        assert int(err.item()) == 0, f"device error word {int(err.item())}"
+        return statistics.mean(ts), statistics.median(ts)
+
+    def line(name, rows, ms, med, alg_bytes, cpu_rows, cpu_s, sample, extra):
+        achieved = alg_bytes / (ms * 1e-3) / 1e9
+        return {"metric": METRIC, "value": rows / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "ms_median": med,
+                "higher_is_better": True, "data": "synthetic",
+                "config": {"workload": name, **extra},
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                             "algorithmic_bytes": alg_bytes},
+                "cpu_baseline": {"value": cpu_rows / cpu_s, "unit": "rows/s", "cores": 1,
+                                 "kind": "oracle", "sample": sample}}
+
+    esize = 2 if cfg.dtype == "bf16" else 4
+    out = []
+    if workload == "verify":
+        d = sdev.gen_config_device(cfg)
+        B, K, V = cfg.B, cfg.K, cfg.V
+        acc = torch.empty((B,), dtype=torch.int32, device=dev)
+        toks = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+        tv = torch.empty((B, K), dtype=torch.float32, device=dev)
+        ms, med = timed(lambda i: lib.sd_verify_reject(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed,
+                                                        i, acc, toks, tv_out=tv, dev_err=err), True)
+        alg = ((2 * K + 1) * V * esize + K * 4 + 4 + (K + 1) * 4 + K * 4) * B
+        h = gen.gen_config_rows(cfg, seqs=list(range(8)))
+        t0 = time.perf_counter()
+        oracle.sd_verify_reject(h["zT"], h["zD"], h["draft"], cfg.tau, cfg.seed, 0)
+        cpu_s = time.perf_counter() - t0
+        out.append(line("verify", B * (K + 1), ms, med, alg, 8 * (K + 1), cpu_s,
+                        "sequences 0-7 of the workload, NumPy fp64, one core",
+                        {"B": B, "K": K, "V": V, "logits": cfg.dtype, "l2": "flushed before each launch"}))
+    else:
+        d = sdev.gen_config_device(cfg)
+        z = d["z"]
+        rows, V, k = z.shape[0], cfg.V, cfg.topk
+        idx = torch.empty((rows, k), dtype=torch.int32, device=dev)
+        sc = torch.empty((rows, k), dtype=torch.float32, device=dev)
+        lp = torch.empty((rows, k), dtype=torch.float32, device=dev)
+        ms, med = timed(lambda i: lib.gumbel_topk(z, k, cfg.tau, cfg.seed, i, idx, score_out=sc,
+                                                  logp_out=lp, dev_err=err), False)
+        alg = rows * (V * esize + k * 12)
+        h = gen.gen_config_rows(cfg, seqs=list(range(16)))
+        t0 = time.perf_counter()
+        oracle.gumbel_topk(h["z"], k, cfg.tau, cfg.seed, 0)
+        cpu_s = time.perf_counter() - t0
+        out.append(line("topk_dense", rows, ms, med, alg, 16, cpu_s,
+                        "rows 0-15 of the workload, NumPy fp64, one core",
+                        {"rows": rows, "V": V, "k": k, "logits": cfg.dtype,
+                         "l2": "inputs (1.2 GB) larger than L2; no flush"}))
+        six, spr = gen.sparse_rows(cfg.seed, rows, cfg.sparse_L, V)
+        ix = torch.from_numpy(six).to(dev)
+        pr = torch.from_numpy(spr.astype(np.float32)).to(dev)
+        ms, med = timed(lambda i: lib.gumbel_topk_sparse(ix, pr, k, cfg.tau, cfg.seed, i, idx,
+                                                         dev_err=err), True)
+        alg = rows * (cfg.sparse_L * 8 + k * 4)
+        t0 = time.perf_counter()
+        oracle.gumbel_topk_sparse(six, spr, k, cfg.tau, cfg.seed, 0)
+        cpu_s = time.perf_counter() - t0
+        out.append(line("topk_sparse", rows, ms, med, alg, rows, cpu_s,
+                        "all rows, NumPy fp64, one core",
+                        {"rows": rows, "L": cfg.sparse_L, "k": k, "l2": "flushed before each launch"}))
+    for o in out:
+        print(json.dumps(o), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -369,7 +470,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sequences", type=int, default=0,
                     help="run B sequences of the workload instead of all 256 (profiling)")
+    ap.add_argument("--workload", choices=[WORKLOAD, "verify", "topk"], default=WORKLOAD,
+                    help="verify / topk: the path's other rows, timed on their own configs (1 GPU)")
     args = ap.parse_args()
+    if args.workload != WORKLOAD:
+        run_rows(args, args.workload)
+        return
     rank, world, local = dist_init()
     try:
         if args.impl == "reference":

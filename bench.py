@@ -31,7 +31,8 @@ METRIC = "verify+resample logit rows/s; achieved HBM TB/s as fraction of B200 pe
 WORKLOAD = "smc_scale"
 
 
-KERNEL_SOURCES = ["resample_online_log_b200/csrc/score.cu", "resample_online_log_b200/csrc/common.cuh"]
+KERNEL_SOURCES = ["resample_online_log_b200/csrc/smc.cu", "resample_online_log_b200/csrc/rows.cuh",
+                  "resample_online_log_b200/csrc/common.cuh"]
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (the measured copy peak is the denominator of frac)
 TRAFFIC_SUMMARY = "profiles/smc_kernel_smc_scale.md"
 

@@ -145,8 +145,9 @@ SMCSD_API sd_status smcsd_resample(const double* logw, int B, int N, uint64_t se
  *                    the call zeroes it first)
  * pt_in, pt_out  device int32 [B, N, P]; must not alias.  -1 = empty slot.
  * ancestors      device int32 [B, N].
- * tok_in/tok_out device int32 [B, N, T] (both or neither); T >= 0.
+ * tok_in/tok_out device int32 [B, N, T] (both or neither; must not overlap); T >= 0.
  * page_refcnt    device int32 [num_pages] or NULL.
+ * Overlapping pt_in / pt_out or tok_in / tok_out ranges -> SD_ERR_INVALID_ARG.
  * Faults: ancestor outside [0, N) -> SD_DEV_ANCESTOR_OOB, that particle's
  *   rows are filled with -1.  Page id outside [0, num_pages) other than -1
  *   -> SD_DEV_PAGE_OOB, copied but not counted.

@@ -106,6 +106,11 @@ def _rows_view(t, lead):
     return V, ld
 
 
+def _check_err(dev_err):
+    """The device error word: a CUDA int32 tensor of one element (or None)."""
+    _want(dev_err, torch.int32, (1,), "dev_err")
+
+
 def _check(name, status):
     if status != SD_OK:
         raise SmcsdError(name, status)
@@ -137,6 +142,7 @@ def smcsd_score(zT, zD, draft_tokens, tau, seed, round, logw_out, bonus_out, log
     _want(tokens_out, torch.int32, (B, N, R), "tokens_out")
     _want(lse_out, torch.float64, (B, N, R, 2), "lse_out")
     _want(lp_out, torch.float64, (B, N, K, 2), "lp_out")
+    _check_err(dev_err)
     st = load().smcsd_score(_p(zT), _p(zD), _dtype(zT), B, N, K, V, ld, _p(draft_tokens),
                             float(tau), int(seed), int(round), _p(logw_prev), _p(logw_out),
                             _p(bonus_out), _p(tv_out), _p(tokens_out), _p(lse_out), _p(lp_out),
@@ -151,6 +157,7 @@ def smcsd_resample(logw, seed, round, ancestors_out, w_out=None, ess_out=None, d
     _want(ancestors_out, torch.int32, (B, N), "ancestors_out")
     _want(w_out, torch.float64, (B, N), "w_out")
     _want(ess_out, torch.float64, (B,), "ess_out")
+    _check_err(dev_err)
     st = load().smcsd_resample(_p(logw), B, N, int(seed), int(round), _p(w_out), _p(ess_out),
                                _p(ancestors_out), _p(dev_err), _stream(stream))
     _check("smcsd_resample", st)
@@ -169,6 +176,7 @@ def kv_pagetable_remap(pt_in, ancestors, pt_out, tok_in=None, tok_out=None, page
         _want(tok_out, torch.int32, (B, N, T), "tok_out")
     if page_refcnt is not None:
         _want(page_refcnt, torch.int32, (num_pages,), "page_refcnt")
+    _check_err(dev_err)
     st = load().kv_pagetable_remap(_p(pt_in), _p(ancestors), B, N, P, _p(pt_out), _p(tok_in), T,
                                    _p(tok_out), _p(page_refcnt), int(num_pages), _p(dev_err),
                                    _stream(stream))
@@ -188,6 +196,7 @@ def sd_verify_reject(zT, zD, draft_tokens, tau, seed, round, accepted_len, out_t
     _want(accepted_len, torch.int32, (B,), "accepted_len")
     _want(out_tokens, torch.int32, (B, R), "out_tokens")
     _want(tv_out, torch.float32, (B, K), "tv_out")
+    _check_err(dev_err)
     st = load().sd_verify_reject(_p(zT), _p(zD), _dtype(zT), B, K, V, ld, _p(draft_tokens),
                                  float(tau), int(seed), int(round), _p(accepted_len),
                                  _p(out_tokens), _p(tv_out), _p(dev_err), _stream(stream))
@@ -201,6 +210,7 @@ def gumbel_topk(z, k, tau, seed, round, idx_out, score_out=None, logp_out=None, 
     _want(idx_out, torch.int32, (rows, k), "idx_out")
     _want(score_out, torch.float32, (rows, k), "score_out")
     _want(logp_out, torch.float32, (rows, k), "logp_out")
+    _check_err(dev_err)
     st = load().gumbel_topk(_p(z), _dtype(z), rows, V, ld, int(k), float(tau), int(seed),
                             int(round), _p(idx_out), _p(score_out), _p(logp_out), _p(dev_err),
                             _stream(stream))
@@ -212,6 +222,7 @@ def gumbel_topk_sparse(idx, prob, k, tau, seed, round, idx_out, dev_err=None, st
     _want(idx, torch.int32, (rows, L), "idx")
     _want(prob, torch.float32, (rows, L), "prob")
     _want(idx_out, torch.int32, (rows, k), "idx_out")
+    _check_err(dev_err)
     st = load().gumbel_topk_sparse(_p(idx), _p(prob), rows, L, int(k), float(tau), int(seed),
                                    int(round), _p(idx_out), _p(dev_err), _stream(stream))
     _check("gumbel_topk_sparse", st)

@@ -6,7 +6,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["abi.cu", "score.cu", "resample.cu", "pagetable.cu", "topk.cu"]
+SOURCES = ["abi.cu", "smc.cu", "verify.cu", "resample.cu", "pagetable.cu", "topk.cu"]
 LIB = os.path.join(HERE, "libsmcsd.so")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]

@@ -81,17 +81,23 @@ extern "C" sd_status kv_pagetable_remap(const int32_t* pt_in, const int32_t* anc
   if ((tok_in == nullptr) != (tok_out == nullptr)) return SD_ERR_INVALID_ARG;
   if (page_refcnt && num_pages < 1) return SD_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  if (page_refcnt && cudaMemsetAsync(page_refcnt, 0, (size_t)num_pages * 4, s) != cudaSuccess)
-    return SD_ERR_CUDA;
-  if (B == 0) return SD_OK;
-  if (!ancestors || !pt_out || (P > 0 && !pt_in)) return SD_ERR_INVALID_ARG;
+  if (B > 0 && (!ancestors || !pt_out || (P > 0 && !pt_in))) return SD_ERR_INVALID_ARG;
   const int64_t particles = (int64_t)B * N;
-  if (P > 0 && pt_in == pt_out) return SD_ERR_INVALID_ARG;
-  if (P > 0) {
+  if (B > 0 && P > 0 && pt_in == pt_out) return SD_ERR_INVALID_ARG;
+  if (B > 0 && P > 0) {
     const int64_t lo_a = (int64_t)(uintptr_t)pt_in, hi_a = lo_a + particles * P * 4;
     const int64_t lo_b = (int64_t)(uintptr_t)pt_out, hi_b = lo_b + particles * P * 4;
     if (lo_a < hi_b && lo_b < hi_a) return SD_ERR_INVALID_ARG;  // must not alias
   }
+  if (B > 0 && tok_in && T > 0) {  // the token gather is out of place too
+    const int64_t lo_a = (int64_t)(uintptr_t)tok_in, hi_a = lo_a + particles * T * 4;
+    const int64_t lo_b = (int64_t)(uintptr_t)tok_out, hi_b = lo_b + particles * T * 4;
+    if (lo_a < hi_b && lo_b < hi_a) return SD_ERR_INVALID_ARG;
+  }
+  // Every argument is checked: only now is anything enqueued.
+  if (page_refcnt && cudaMemsetAsync(page_refcnt, 0, (size_t)num_pages * 4, s) != cudaSuccess)
+    return SD_ERR_CUDA;
+  if (B == 0) return SD_OK;
   const int vec = (P % 4 == 0) && ((uintptr_t)pt_in % 16 == 0) && ((uintptr_t)pt_out % 16 == 0);
   const int threads = 256;
   const int64_t blocks = (particles * 32 + threads - 1) / threads;

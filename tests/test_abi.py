@@ -63,6 +63,8 @@ def test_host_argument_checks_need_no_gpu():
                                 None) == lib.SD_ERR_INVALID_ARG     # tok_in without tok_out
     assert L.kv_pagetable_remap(vp(16), vp(16), 1, 1, 4, vp(16), None, 0, None, None, 0, None,
                                 None) == lib.SD_ERR_INVALID_ARG     # aliasing pt_in / pt_out
+    assert L.kv_pagetable_remap(vp(16), vp(16), 1, 2, 4, vp(4096), vp(256), 3, vp(264), None, 0,
+                                None, None) == lib.SD_ERR_INVALID_ARG  # overlapping tok_in / tok_out
     assert L.sd_verify_reject(vp(1), vp(1), 1, 1, 0, 10, 10, vp(1), 1.0, 0, 0, vp(1), vp(1), None,
                               None, None) == lib.SD_ERR_INVALID_ARG  # K = 0
     assert L.gumbel_topk(vp(1), 1, 1, 10, 10, 11, 1.0, 0, 0, vp(1), None, None, None,
@@ -78,3 +80,16 @@ def test_product_path_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_binding_rejects_a_bad_error_word():
+    """The error word is written by the kernels: a host tensor or a wrong dtype or
+    size is refused before the library is called."""
+    import torch
+    with pytest.raises(ValueError):
+        lib._check_err(torch.zeros((1,), dtype=torch.int32))          # not on a GPU
+    with pytest.raises(ValueError):
+        lib._check_err(torch.zeros((2,), dtype=torch.int32))
+    with pytest.raises(ValueError):
+        lib._check_err(torch.zeros((1,), dtype=torch.float32))
+    lib._check_err(None)

@@ -163,56 +163,138 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
-def _oracle_sequence(cfg, b):
+def _oracle_inputs(cfg, b, parts):
+    """Host inputs of particles `parts` of sequence b of the workload (the seeded
+    generator's exact values) and that sequence's page table."""
     from synth import gen
-    h = gen.gen_config_rows(cfg, seqs=[b])
-    pt = gen.page_table(cfg.seed, cfg.B, cfg.N, cfg.P)[b:b + 1]
-    return h, pt
+    rows = np.array([(b * cfg.N + n) * cfg.R + k for n in parts for k in range(cfg.R)])
+    zt, zd = gen.gen_rows(cfg.seed, rows, cfg.V, cfg.sigma_z, cfg.L_head,
+                          np.full(rows.shape, cfg.sigma_d_of_seq(b), dtype=np.float32), cfg.dtype)
+    P, R = len(parts), cfg.R
+    zt = zt.reshape(1, P, R, cfg.V)
+    zd = zd.reshape(1, P, R, cfg.V)
+    did = rows.reshape(P, R)[:, :cfg.K].reshape(-1)
+    x = gen.draft_tokens_for_rows(cfg.seed, did, zd[:, :, :cfg.K].reshape(-1, cfg.V), cfg.tau)
+    pt = gen.page_table(cfg.seed, cfg.B, cfg.N, cfg.P)[b:b + 1, parts]
+    return dict(zT=zt, zD=zd, draft=x.reshape(1, P, cfg.K)), pt
 
 
-def _oracle_round(cfg, h, pt, parts):
-    """The oracle's SMC-SD round on particles `parts` of one sequence."""
+def _oracle_round(cfg, h, pt):
+    """The oracle's SMC-SD round (score -> resample -> remap) on the given particles."""
     import oracle
-    zT, zD, x = h["zT"][:, parts], h["zD"][:, parts], h["draft"][:, parts]
-    o = oracle.smcsd_score(zT, zD, x, cfg.tau, cfg.seed, 1)
+    o = oracle.smcsd_score(h["zT"], h["zD"], h["draft"], cfg.tau, cfg.seed, 1)
     r = oracle.smcsd_resample(o["logw"], cfg.seed, 1)
-    p = pt[:, parts]
-    oracle.kv_pagetable_remap(p, r["ancestors"], num_pages=int(pt.size), tok_in=o["tokens"])
-    return len(parts) * cfg.R
+    oracle.kv_pagetable_remap(pt, r["ancestors"], num_pages=cfg.B * cfg.N * cfg.P,
+                              tok_in=o["tokens"])
+    return h["zT"].shape[1] * cfg.R
+
+
+PARTS_PER_TASK = 8  # particles of one sequence per oracle process (72 row pairs)
+
+
+def _oracle_proc(conn, b, n0):
+    """One host core: generates its particles of the workload once, then runs the
+    oracle's round on them on request, `reps` times or until `budget_s` seconds of
+    compute, and answers (row pairs, seconds)."""
+    from synth import gen
+    cfg = gen.CONFIGS[WORKLOAD]
+    h, pt = _oracle_inputs(cfg, b, list(range(n0, n0 + PARTS_PER_TASK)))
+    conn.send("ready")
+    while True:
+        msg = conn.recv()
+        if msg is None:
+            break
+        reps, budget_s = msg
+        rows, t = 0, 0.0
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            rows += _oracle_round(cfg, h, pt)
+            t += time.perf_counter() - t0
+            if budget_s and t >= budget_s:
+                break
+        conn.send((rows, t))
+    conn.close()
+
+
+def oracle_cores():
+    """Host cores the oracle baseline uses: all this process may run on (at most 32)."""
+    return max(1, min(32, len(os.sched_getaffinity(0))))
+
+
+class OracleCores:
+    """One spawned process per host core, each holding 8 particles of its own
+    sequence of the workload (process w: sequence w // 4, particles 8 (w % 4) ..)."""
+
+    def __init__(self, cfg, workers):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        per_seq = cfg.N // PARTS_PER_TASK
+        self.conns, self.procs = [], []
+        for w in range(workers):
+            a, c = ctx.Pipe()
+            pr = ctx.Process(target=_oracle_proc,
+                             args=(c, w // per_seq, (w % per_seq) * PARTS_PER_TASK), daemon=True)
+            pr.start()
+            self.conns.append(a)
+            self.procs.append(pr)
+        for a in self.conns:
+            assert a.recv() == "ready"
+
+    def run(self, reps, budget_s=0.0):
+        for a in self.conns:
+            a.send((reps, budget_s))
+        return [a.recv() for a in self.conns]
+
+    def close(self):
+        for a in self.conns:
+            a.send(None)
+        for pr in self.procs:
+            pr.join(timeout=30)
 
 
 def oracle_baseline(cfg, budget_s=10.0):
-    """Times the oracle (as it stands, one host core) on one whole sequence of the
-    workload, repeated until the budget is used; returns rows/s, seconds, runs."""
-    h, pt = _oracle_sequence(cfg, 0)
-    rows, t_total, runs = 0, 0.0, 0
-    while runs == 0 or t_total < budget_s:
-        t0 = time.perf_counter()
-        rows += _oracle_round(cfg, h, pt, list(range(cfg.N)))
-        t_total += time.perf_counter() - t0
-        runs += 1
-    return rows / t_total, t_total, runs
+    """The oracle (as it stands) on every host core at once, each core on 8
+    particles of its own sequence of the workload until `budget_s` seconds of
+    compute; returns (row pairs/s of all cores together = total rows / the
+    slowest core's time, cores, sample text)."""
+    workers = oracle_cores()
+    pool = OracleCores(cfg, workers)
+    try:
+        pool.run(1)  # warm
+        res = pool.run(10 ** 6, budget_s)
+    finally:
+        pool.close()
+    rows = sum(r for r, _ in res)
+    t = max(s for _, s in res)
+    sample = (f"{workers} processes x {PARTS_PER_TASK} particles x {cfg.R} row pairs "
+              f"(V={cfg.V}) of the workload, {rows} row pairs, {t:.1f} s on the slowest core")
+    return rows / t, workers, sample
 
 
 def run_reference(args, rank, world):
-    """--impl reference: the fp64 NumPy oracle on a host core (rank 0 only).
-    One step = the oracle's round on 8 particles (72 row pairs) of one sequence."""
+    """--impl reference: the fp64 NumPy oracle on the host cores (rank 0 only).
+    One step = the oracle's round on 8 particles (72 row pairs) per core, every
+    core at once on its own particles of the workload."""
     if rank != 0:
         return
     from synth import gen
     cfg = gen.CONFIGS[WORKLOAD]
-    h, pt = _oracle_sequence(cfg, 0)
-    groups = [list(range(g, g + 8)) for g in range(0, cfg.N, 8)]
-    for i in range(args.warmup):
-        _oracle_round(cfg, h, pt, groups[i % len(groups)])
-    rows, t_total = 0, 0.0
-    for i in range(args.steps):
-        t0 = time.perf_counter()
-        rows += _oracle_round(cfg, h, pt, groups[i % len(groups)])
-        t_total += time.perf_counter() - t0
+    workers = oracle_cores()
+    pool = OracleCores(cfg, workers)
+    try:
+        for i in range(args.warmup):
+            pool.run(1)
+        rows, t_total = 0, 0.0
+        for i in range(args.steps):
+            t0 = time.perf_counter()
+            res = pool.run(1)
+            t_total += time.perf_counter() - t0
+            rows += sum(r for r, _ in res)
+    finally:
+        pool.close()
     value = rows / t_total
-    sample = (f"per step 8 particles x {cfg.R} row pairs (V={cfg.V}) of sequence 0 of the "
-              f"workload, NumPy fp64, one core")
+    sample = (f"per step {workers} processes x {PARTS_PER_TASK} particles x {cfg.R} row pairs "
+              f"(V={cfg.V}) of the workload, NumPy fp64")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -220,7 +302,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": cfg.B, "N": cfg.N, "K": cfg.K, "V": cfg.V,
                    "logits": cfg.dtype, "sample": sample},
-        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": workers, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -351,10 +433,9 @@ def run_ours(args, rank, world, local):
                        "steps": args.e2e_steps}
         del h_zT, h_zD
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, t, runs = oracle_baseline(gen.CONFIGS[WORKLOAD], budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle",
-                                "sample": f"sequence 0 of the workload ({N * R} row pairs) x "
-                                          f"{runs} run(s), {t:.1f} s of CPU"}
+        v, cores, sample = oracle_baseline(gen.CONFIGS[WORKLOAD], budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -14,9 +14,10 @@ constexpr float kGumbelMinF = -2.8104283f;   // -log(24 log 2), rounded down
 constexpr float kGumbelMaxF = 16.635532f;    // -log(-log1p(-2^-24)), rounded up
 constexpr double kGumbelMin = -2.8104282144774236;
 
-// Iteration limit of every spin-wait on an mbarrier; past it the kernel
-// records SD_DEV_TIMEOUT and carries on with whatever the buffer holds.
-constexpr uint32_t kWaitLimit = 1u << 24;
+// Every wait on an mbarrier is bounded in time (read from %globaltimer): past
+// kWaitNs of waiting the kernel records SD_DEV_TIMEOUT and carries on with
+// whatever the buffer holds.
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 
 // ---------------------------------------------------------------- Philox4x32-10
 // Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3"
@@ -142,11 +143,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false if the phase did not complete within kWaitLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: false if the phase did not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-  return false;
+    if ((i & 15u) == 0 && globaltimer_ns() - t0 >= limit_ns) return false;
+  }
 }
 
 // Bulk (non-tensor) copy global -> this CTA's shared memory, completing on an

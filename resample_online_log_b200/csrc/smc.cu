@@ -78,14 +78,21 @@ enum WaitSite : uint32_t {
   kWsAdone = 1u << 13, kWsBook = 1u << 14, kWsBmsg = 1u << 15
 };
 
-// Bounded wait; after one expiry every later wait of the CTA returns at once
-// (the outputs are then garbage, SD_DEV_TIMEOUT is set, nothing hangs).
+// Bounded wait (kWaitNs of polling).  After one expiry every later abortable
+// wait of the CTA returns at once (outputs are then garbage, SD_DEV_TIMEOUT is
+// set, nothing hangs).  The waits that order the bulk copies into the ring are
+// not abortable: a stage is refilled only after every producer has seen its
+// last copy land, so no copy can still be in flight into a CTA that finishes.
 __device__ __forceinline__ void swait(uint64_t* bar, uint32_t parity, SmcTail* tl, uint32_t* err,
-                                      uint32_t site) {
+                                      uint32_t site, bool abortable = true) {
   if (mbar_try_wait(bar, parity)) return;
   volatile int* ab = &tl->abort_flag;
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if ((i & 15u) == 0 && *ab) return;  // (a shared-memory read every 16 polls only)
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if ((i & 15u) == 0) {  // (the abort flag and the clock every 16 polls only)
+      if (abortable && *ab) return;
+      if (globaltimer_ns() - t0 >= kWaitNs) break;
+    }
     if (mbar_try_wait(bar, parity)) return;
   }
   *ab = 1;
@@ -501,7 +508,7 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
     for (int it = 0; it <= nrows; ++it) {
       if (it < nrows) {  // row it: refill its stage once read, then its message
         if (it + nS < nrows) {
-          swait(&tl->empty[stage], (uint32_t)((it / nS) & 1), tl, a.dev_err, kWsAfull);
+          swait(&tl->empty[stage], (uint32_t)((it / nS) & 1), tl, a.dev_err, kWsAfull, false);
           if (lane == 0) issue(it + nS, stage);
         }
         swait(&tl->afull[it & 1], (uint32_t)((it >> 1) & 1), tl, a.dev_err, kWsAfull);
@@ -684,7 +691,7 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       }
       x_next = (it + 1 < nrows && kn < a.K) ? a.draft[un * a.K + kn] : -1;
     }
-    swait(&tl->full[stage], phase, tl, a.dev_err, kWsFull);
+    swait(&tl->full[stage], phase, tl, a.dev_err, kWsFull, false);
     const int64_t row = unit * a.R + k;
     const TIn* stT = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb);
     const TIn* stD = reinterpret_cast<const TIn*>(smem + (size_t)stage * 2 * sb + sb);

@@ -6,16 +6,16 @@
 // parallel; item 1: the logit n-gram store keeps only the top-10 (index,
 // probability) pairs of a row, unstored entries having probability 0.
 //
-// Dense kernel (one CTA per row, one streaming pass over HBM):
-//   * online log-sum-exp of s = z / tau (one exp2 per entry) for the log-probs;
-//   * a per-thread list of its best k+1 perturbed scores s_v + g_v under a
-//     pruning threshold T that is always a lower bound on the row's (k+1)-th
-//     best score (a thread's own (k+1)-th best, raised through a CTA-shared
-//     maximum).  Groups of four entries with s + g_max < T skip the Philox call;
-//     an entry with u <= 1 - e^{s - T} cannot reach T (e^{-y} >= 1 - y) and
-//     skips the logs;
-//   * the fp32 scores carry error bounds; when the order of the first k+1 is
-//     not settled by them, the row is re-scored exactly in fp64.
+// Dense kernel (persistent CTAs, two per SM, each taking rows in turn): the
+// row is read twice, the second time from L2 (the first read asks L2 to keep
+// it) -- once for the log-sum-exp and each thread's largest logit, whose
+// exact perturbed scores give a lower bound T on the row's k-th best score;
+// once for the candidates under T: four entries whose s + g_max < T skip the
+// Philox call, an entry with u <= 1 - e^{s - T} cannot reach T (e^{-y} >=
+// 1 - y) and skips the logs.  The fp32 scores carry error bounds; when the
+// order of the first k+1 is not settled by them, the row is re-scored exactly
+// in fp64.
+#include <algorithm>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -62,23 +62,22 @@ __device__ __forceinline__ float ld_elem<uint16_t>(const uint16_t* p, int i) {
   return __uint_as_float((uint32_t)p[i] << 16);
 }
 
-// Inserts (s, d, v) into a descending list of length L (ties to the lower v);
-// returns the upper bound of the entry pushed out (or -inf).
-template <int L>
-__device__ __forceinline__ float list_insert(float (&ls)[L], float (&ld)[L], int (&li)[L], float s,
-                                             float d, int v) {
-#pragma unroll
-  for (int j = 0; j < L; ++j) {
-    const bool before = s > ls[j] || (s == ls[j] && v < li[j]);
-    if (before) {
-      const float ts = ls[j], td = ld[j];
-      const int ti = li[j];
-      ls[j] = s;
-      ld[j] = d;
-      li[j] = v;
-      s = ts;
-      d = td;
-      v = ti;
+// Inserts (s, d, v) into a descending list of length n held in a column of
+// shared memory (entry j at j * stride; ties to the lower v); returns the upper
+// bound of the entry pushed out (or -inf).
+__device__ __forceinline__ float list_insert_col(float* ls, float* ld, int* li, int stride, int n,
+                                                 float s, float d, int v) {
+  for (int j = 0; j < n; ++j) {
+    const float bs = ls[j * stride];
+    const int bi = li[j * stride];
+    if (s > bs || (s == bs && v < bi)) {
+      const float bd = ld[j * stride];
+      ls[j * stride] = s;
+      ld[j * stride] = d;
+      li[j * stride] = v;
+      s = bs;
+      d = bd;
+      v = bi;
     }
   }
   return v == 0x7FFFFFFF ? -INFINITY : s + d;
@@ -165,219 +164,396 @@ __device__ __noinline__ void exact_topk_row(const TIn* row, int V, int k1, float
   }
 }
 
+// Eight consecutive entries of a row (one 16-byte chunk of bf16, two of fp32)
+// as floats; entries at or past V read as -inf.  `hint` is the L2 policy of
+// the vector loads.  The raw form (load8_raw, then unpack8) lets a thread keep
+// several chunks in flight.
+template <typename TIn>
+__device__ __forceinline__ void load8(const TIn* row, int v0, int V, bool vec, uint64_t hint,
+                                      float* z);
+template <>
+__device__ __forceinline__ void load8<uint16_t>(const uint16_t* row, int v0, int V, bool vec,
+                                                uint64_t hint, float* z) {
+  if (vec && v0 + 8 <= V) {
+    const uint4 u = ldg_hint(row + v0, hint);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      z[2 * j] = __uint_as_float(w[j] << 16);
+      z[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) z[j] = v0 + j < V ? ld_elem<uint16_t>(row, v0 + j) : -INFINITY;
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* row, int v0, int V, bool vec,
+                                             uint64_t hint, float* z) {
+  if (vec && v0 + 8 <= V) {
+    const uint4 a = ldg_hint(row + v0, hint), b = ldg_hint(row + v0 + 4, hint);
+    z[0] = __uint_as_float(a.x); z[1] = __uint_as_float(a.y);
+    z[2] = __uint_as_float(a.z); z[3] = __uint_as_float(a.w);
+    z[4] = __uint_as_float(b.x); z[5] = __uint_as_float(b.y);
+    z[6] = __uint_as_float(b.z); z[7] = __uint_as_float(b.w);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) z[j] = v0 + j < V ? row[v0 + j] : -INFINITY;
+  }
+}
+
+template <typename TIn>
+struct Raw8 {
+  uint4 a, b;  // bf16: a only
+};
+template <typename TIn>
+__device__ __forceinline__ Raw8<TIn> load8_raw(const TIn* row, int v0, int V, bool vec,
+                                               uint64_t hint) {
+  Raw8<TIn> r;
+  if (vec && v0 + 8 <= V) {
+    r.a = ldg_hint(row + v0, hint);
+    if (sizeof(TIn) == 4) r.b = ldg_hint(row + v0 + 4, hint);
+  } else {
+    float zz[8];
+    load8<TIn>(row, v0, V, false, hint, zz);
+    if (sizeof(TIn) == 2) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[j] = (__float_as_uint(zz[2 * j]) >> 16) | (__float_as_uint(zz[2 * j + 1]) & 0xFFFF0000u);
+      r.a = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      r.a = make_uint4(__float_as_uint(zz[0]), __float_as_uint(zz[1]), __float_as_uint(zz[2]),
+                       __float_as_uint(zz[3]));
+      r.b = make_uint4(__float_as_uint(zz[4]), __float_as_uint(zz[5]), __float_as_uint(zz[6]),
+                       __float_as_uint(zz[7]));
+    }
+  }
+  return r;
+}
+template <typename TIn>
+__device__ __forceinline__ void unpack8(const Raw8<TIn>& r, float* z) {
+  if (sizeof(TIn) == 2) {
+    const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      z[2 * j] = __uint_as_float(w[j] << 16);
+      z[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else {
+    z[0] = __uint_as_float(r.a.x); z[1] = __uint_as_float(r.a.y);
+    z[2] = __uint_as_float(r.a.z); z[3] = __uint_as_float(r.a.w);
+    z[4] = __uint_as_float(r.b.x); z[5] = __uint_as_float(r.b.y);
+    z[6] = __uint_as_float(r.b.z); z[7] = __uint_as_float(r.b.w);
+  }
+}
+constexpr int kTopkUnroll = 4;   // chunks a thread has in flight in the first pass
+
+// The k-th largest of one value per thread of the CTA (-inf if fewer than k
+// are finite): k rounds of warp maxima, each removing one winning lane, then
+// the same over the warps' k best.
+__device__ __noinline__ float cta_kth_largest(float v, int k, float* buf /* [nwarps * k] */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int r = 0; r < k; ++r) {
+    float w = v;
+    asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(w));
+    const unsigned hit = __ballot_sync(0xffffffffu, v == w && w > -INFINITY);
+    if (hit && lane == __ffs(hit) - 1) v = -INFINITY;
+    if (lane == 0) buf[warp * k + r] = hit ? w : -INFINITY;
+  }
+  __syncthreads();
+  float res = -INFINITY;
+  if (warp == 0) {
+    const int n = nw * k;  // <= 16 * 16: at most 8 per lane
+    float h[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = lane + 32 * i < n ? buf[lane + 32 * i] : -INFINITY;
+    for (int r = 0; r < k; ++r) {
+      float m = h[0];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) m = fmaxf(m, h[i]);
+      float w = m;
+      asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(w));
+      const unsigned hit = __ballot_sync(0xffffffffu, m == w && w > -INFINITY);
+      if (hit && lane == __ffs(hit) - 1) {
+        bool done = false;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (!done && h[i] == w) {
+            h[i] = -INFINITY;
+            done = true;
+          }
+      }
+      res = hit ? w : -INFINITY;
+    }
+    if (lane == 0) buf[0] = res;
+  }
+  __syncthreads();
+  res = buf[0];
+  __syncthreads();
+  return res;
+}
+
+// Dense rows.  A persistent CTA takes rows in turn and reads each twice:
+//   pass 1 (HBM, kept in L2 with an evict-last hint): the row's log-sum-exp
+//     (one exp2 per entry, online per thread) and each thread's largest logit;
+//   threshold: the exact fp32 perturbed scores of those per-thread maxima
+//     (one Philox word each, minus their error bound) -- the k-th largest of
+//     them is a lower bound T on the row's k-th best score;
+//   pass 2 (L2): groups of four entries that even g_max cannot lift to T skip
+//     the Philox call; an entry whose word proves u <= 1 - e^{s - T} (an
+//     integer leading-bit test first, then the exp2) cannot reach T and skips
+//     the logs; the rest enter the thread's descending list of k+1 candidates
+//     with fp32 error bounds.
+// The lists merge into the first k+1 ranks; when the fp32 bounds do not settle
+// their order, the row is re-scored exactly in fp64.
 template <typename TIn, int L>
-__global__ void __launch_bounds__(kTopkThreads) topk_dense_kernel(
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_dense_kernel(
     const TIn* __restrict__ z, int rows, int V, int64_t ld, int k, float inv_tau, double tau64,
     uint64_t seed, uint64_t round, int vec, int32_t* __restrict__ idx_out, float* score_out,
     float* logp_out, uint32_t* dev_err) {
   __shared__ TopkSmem sm;
-  const int r = blockIdx.x;
+  __shared__ float kbuf[(kTopkThreads / 32) * kTopkMax];
+  extern __shared__ float lists[];  // [3][L][blockDim.x]: scores, error bounds, indices
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x;
   const int k1 = k + 1;
-  const TIn* row = z + (int64_t)r * ld;
   const Stream st(seed, round, SD_STREAM_TOPK_DENSE);
-  if (tid == 0) {
-    sm.thr = f2ord(-INFINITY);
-    sm.dropped = f2ord(-INFINITY);
-    sm.ncand = 0;
-    sm.flag = 0;
-  }
-  __syncthreads();
+  const PhiloxKeys K = philox_keys(seed);
+  const float cT = kLog2e * inv_tau;  // log2(e) / tau
+  const int nchunks = (V + 7) / 8;
+  const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+  const bool vecok = vec != 0;
 
-  float ls[L], ldv[L];
-  int li[L];
-  float dropped_hi = -INFINITY;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const TIn* row = z + (int64_t)r * ld;
+    const uint32_t rid = (uint32_t)r;
+    if (tid == 0) {
+      sm.thr = f2ord(-INFINITY);
+      sm.dropped = f2ord(-INFINITY);
+      sm.ncand = 0;
+      sm.flag = 0;
+    }
+    __syncthreads();
+    // ---------------- pass 1: log-sum-exp and per-thread maxima
+    float m = -INFINITY, S = 0.f, zmax = -INFINITY;
+    int zarg = 0x7FFFFFFF;
+    bool bad = false;
+    for (int c0 = tid; c0 < nchunks; c0 += kTopkUnroll * nthr) {
+     Raw8<TIn> raw[kTopkUnroll];
 #pragma unroll
-  for (int j = 0; j < L; ++j) {
-    ls[j] = -INFINITY;
-    ldv[j] = 0.f;
-    li[j] = 0x7FFFFFFF;
-  }
-  float T = -INFINITY;        // lower bound on the row's (k+1)-th best score
-  float m = -INFINITY, S = 0.f;
-  bool bad = false;
-  constexpr int EPC = 8;      // entries per chunk (two Philox groups)
-  const int nchunks = (V + EPC - 1) / EPC;
-  int iter = 0;
-  for (int c = tid; c < nchunks; c += nthr, ++iter) {
-    const int v0 = c * EPC;
-    float s[EPC];
-    if (vec && v0 + EPC <= V) {
-      if (sizeof(TIn) == 2) {
-        const uint4 u = *reinterpret_cast<const uint4*>(row + v0);
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+     for (int u = 0; u < kTopkUnroll; ++u)
+       if (c0 + u * nthr < nchunks) raw[u] = load8_raw<TIn>(row, (c0 + u * nthr) * 8, V, vecok, keep);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          s[2 * j] = __uint_as_float(w4[j] << 16) * inv_tau;
-          s[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u) * inv_tau;
-        }
-      } else {
-        const float4 a = *reinterpret_cast<const float4*>(row + v0);
-        const float4 b = *reinterpret_cast<const float4*>(row + v0 + 4);
-        s[0] = a.x * inv_tau; s[1] = a.y * inv_tau; s[2] = a.z * inv_tau; s[3] = a.w * inv_tau;
-        s[4] = b.x * inv_tau; s[5] = b.y * inv_tau; s[6] = b.z * inv_tau; s[7] = b.w * inv_tau;
+     for (int u = 0; u < kTopkUnroll; ++u) {
+      const int c = c0 + u * nthr;
+      if (c >= nchunks) break;
+      float zz[8];
+      unpack8<TIn>(raw[u], zz);
+      float cm = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cm = fmaxf(cm, zz[j]);
+      if (cm > zmax) {
+        zmax = cm;
+#pragma unroll
+        for (int j = 7; j >= 0; --j)
+          if (zz[j] == cm) zarg = c * 8 + j;
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < EPC; ++j) s[j] = v0 + j < V ? ld_elem<TIn>(row, v0 + j) * inv_tau : -INFINITY;
-    }
-    // online log-sum-exp (entries relative to the running max)
-    float cm = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < EPC; ++j) {
-      cm = fmaxf(cm, s[j]);
-      bad |= (s[j] != s[j]) || (s[j] == INFINITY);
-    }
-    if (cm > m) {
-      S = (m == -INFINITY) ? 0.f : S * ex2((m - cm) * kLog2e);
-      m = cm;
-    }
-    if (m > -INFINITY) {
-#pragma unroll
-      for (int j = 0; j < EPC; ++j) S += ex2((s[j] - m) * kLog2e);
-    }
-    // candidates
-#pragma unroll
-    for (int gq = 0; gq < 2; ++gq) {
-      const float gm = fmaxf(fmaxf(s[4 * gq], s[4 * gq + 1]), fmaxf(s[4 * gq + 2], s[4 * gq + 3]));
-      if (!(gm + kGumbelMaxF + 1e-4f + 1e-6f * fabsf(gm) >= T)) continue;
-      const U4 w = st.at((uint32_t)((v0 >> 2) + gq), (uint32_t)r);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float sv = s[4 * gq + j];
-        if (!(sv > -INFINITY)) continue;
-        const float u = uniform_f32(word_of(w, j));
-        if (T > -INFINITY) {
-          const float y = ex2((sv - T) * kLog2e) * 1.001f + 1e-30f;
-          if (u < (1.0f - y) - 2.4e-7f) continue;
-        }
-        const float g32 = gumbel_f32(u);
-        const float sc = sv + g32;
-        const float d = score_err(sv, g32);
-        if (!(sc + d >= T)) continue;
-        dropped_hi = fmaxf(dropped_hi, list_insert<L>(ls, ldv, li, sc, d, v0 + 4 * gq + j));
-        float kth = -INFINITY;  // lower bound of this thread's (k+1)-th best (-inf until held)
-#pragma unroll
-        for (int t = 0; t < L; ++t)
-          if (t == k1 - 1) kth = ls[t] - ldv[t];
-        T = fmaxf(T, kth);
+      if (cm > m) {
+        S = (m == -INFINITY) ? 0.f : S * ex2((m - cm) * cT);
+        m = cm;
       }
+      if (m > -INFINITY) {
+        const float nm = -m * cT;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) S += ex2(fmaf(zz[j], cT, nm));
+      }
+     }
     }
-    if ((iter & 3) == 3) {  // share / refresh the CTA threshold
-      atomicMax(&sm.thr, f2ord(T));
-      T = fmaxf(T, ord2f(*(volatile int*)&sm.thr));
-    }
-  }
-  atomicMax(&sm.thr, f2ord(T));
-  atomicMax(&sm.dropped, f2ord(dropped_hi));
-
-  // lse: CTA combine of (m, S)
-  float M = warp_max(m);
-  float Sw = (m == -INFINITY) ? 0.f : S * ex2((m - M) * kLog2e);
-  Sw = warp_sum(Sw);
-  if (lane == 0) {
-    sm.red_m[warp] = M;
-    sm.red_s[warp] = Sw;
-  }
-  const int badw = __any_sync(0xffffffffu, bad);
-  if (badw && lane == 0) atomicOr(&sm.flag, 1);
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = nthr >> 5;
-    const float pm = lane < nw ? sm.red_m[lane] : -INFINITY;
-    const float ps = lane < nw ? sm.red_s[lane] : 0.f;
-    const float MM = warp_max(pm);
-    const double t = (lane < nw && pm > -INFINITY) ? (double)ps * (double)ex2((pm - MM) * kLog2e) : 0.0;
-    const double SS = warp_sum_d(t);
+    // lse: CTA combine of (m, S) in fp64
+    // a NaN entry leaves S NaN (its exp2 is NaN), a +inf entry makes m +inf
+    bad = m == INFINITY || S != S;
+    float M = warp_max(m);
+    float Sw = (m == -INFINITY) ? 0.f : S * ex2((m - M) * cT);
+    Sw = warp_sum(Sw);
     if (lane == 0) {
-      sm.lse = (double)MM + log(SS);
-      if (!(MM > -INFINITY)) sm.flag |= 1;  // all -inf
+      sm.red_m[warp] = M;
+      sm.red_s[warp] = Sw;
     }
-  }
-  // gather the list entries that can still make the top k+1
-  const float Tfin = ord2f(sm.thr);
-#pragma unroll
-  for (int j = 0; j < L; ++j) {
-    if (li[j] != 0x7FFFFFFF && ls[j] + ldv[j] >= Tfin) {
-      const int pos = atomicAdd(&sm.ncand, 1);
-      if (pos < kCandCap) {
-        sm.cs[pos] = ls[j];
-        sm.cd[pos] = ldv[j];
-        sm.ci[pos] = li[j];
-      }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&sm.flag, 1);
+    // threshold: exact fp32 lower bounds of the per-thread maxima's perturbed scores
+    float lo = -INFINITY;
+    if (zarg != 0x7FFFFFFF) {
+      const U4 w = philox_rk((uint32_t)(zarg >> 2), rid, st.c2, st.c3, K);
+      const float a32 = zmax * inv_tau;
+      const float g32 = gumbel_f32(uniform_f32(word_of(w, zarg & 3)));
+      lo = a32 + g32 - score_err(a32, g32);
     }
-  }
-  __syncthreads();
-  if (sm.flag & 1) {  // non-finite row
-    if (tid < k) {
-      idx_out[(int64_t)r * k + tid] = -1;
-      if (score_out) score_out[(int64_t)r * k + tid] = NAN;
-      if (logp_out) logp_out[(int64_t)r * k + tid] = NAN;
-    }
-    if (tid == 0) raise_err(dev_err, SD_DEV_NONFINITE);
-    return;
-  }
-  const int n = min(sm.ncand, kCandCap);
-  bool need_exact = sm.ncand > kCandCap;
-  // warp 0 extracts the top k+1 (descending, ties to the lower index)
-  if (warp == 0) {
-    bool ambiguous = false;
-    float prev_lo = INFINITY;
-    for (int rnk = 0; rnk < k1; ++rnk) {
-      float bs = -INFINITY, bd = 0.f;
-      int bi = 0x7FFFFFFF, bp = -1;
-      for (int p = lane; p < n; p += 32) {
-        const float s = sm.cs[p];
-        const int v = sm.ci[p];
-        if (s > bs || (s == bs && v < bi)) {
-          bs = s;
-          bi = v;
-          bd = sm.cd[p];
-          bp = p;
-        }
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        const float od = __shfl_xor_sync(0xffffffffu, bd, o);
-        const int op = __shfl_xor_sync(0xffffffffu, bp, o);
-        if (os > bs || (os == bs && oi < bi)) {
-          bs = os;
-          bi = oi;
-          bd = od;
-          bp = op;
-        }
-      }
-      // the order between this rank and the previous one must be settled
-      if (rnk > 0 && bi != 0x7FFFFFFF && !(bs + bd < prev_lo)) ambiguous = true;
-      // nothing evicted from a thread's list may reach the k-th output
-      if (rnk == k - 1 && !(ord2f(sm.dropped) < bs - bd)) ambiguous = true;
-      prev_lo = bs - bd;
+    __syncthreads();
+    if (warp == 0) {
+      const int nw = nthr >> 5;
+      const float pm = lane < nw ? sm.red_m[lane] : -INFINITY;
+      const float ps = lane < nw ? sm.red_s[lane] : 0.f;
+      const float MM = warp_max(pm);
+      const double t = (lane < nw && pm > -INFINITY) ? (double)ps * (double)ex2((pm - MM) * cT) : 0.0;
+      const double SS = warp_sum_d(t);
       if (lane == 0) {
-        sm.s64[rnk] = bs;
-        sm.i64[rnk] = bi;
-        if (bp >= 0) sm.cs[bp] = -INFINITY;
+        sm.lse = (double)MM / tau64 + log(SS);
+        if (!(MM > -INFINITY)) sm.flag |= 1;  // all -inf
       }
-      __syncwarp();
     }
-    if (lane == 0 && ambiguous) sm.flag |= 2;
-  }
-  __syncthreads();
-  need_exact = need_exact || (sm.flag & 2);
-  if (need_exact) {
-    // lo bound of the k-th candidate: everything that can reach it is re-scored
-    const float lo_k = (float)sm.s64[k - 1] - 1e-3f - 1e-5f * fabsf((float)sm.s64[k - 1]);
+    const float T0 = cta_kth_largest(lo, k, kbuf);  // (syncs the CTA)
+    const bool rowbad = (sm.flag & 1) != 0;
+
+    // ---------------- pass 2: the candidates
+    // this thread's descending list of its best k+1 candidates, in a column of
+    // shared memory (insertions are rare: registers stay with the stream)
+    float* ls = lists + tid;
+    float* ldv = lists + L * nthr + tid;
+    int* li = reinterpret_cast<int*>(lists + 2 * L * nthr) + tid;
+    float dropped_hi = -INFINITY;
+    for (int j = 0; j < L; ++j) {
+      ls[j * nthr] = -INFINITY;
+      ldv[j * nthr] = 0.f;
+      li[j * nthr] = 0x7FFFFFFF;
+    }
+    float T = T0;
+    if (!rowbad && tid < nchunks) {
+      Raw8<TIn> nxt = load8_raw<TIn>(row, tid * 8, V, vecok, drop);
+      for (int c = tid; c < nchunks; c += nthr) {
+        const Raw8<TIn> cur = nxt;
+        if (c + nthr < nchunks) nxt = load8_raw<TIn>(row, (c + nthr) * 8, V, vecok, drop);
+        float zz[8];
+        unpack8<TIn>(cur, zz);
+#pragma unroll 1
+        for (int gq = 0; gq < 2; ++gq) {  // one Philox block: four entries
+          float z4[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) z4[j] = gq ? zz[4 + j] : zz[j];
+          const float zm = fmaxf(fmaxf(z4[0], z4[1]), fmaxf(z4[2], z4[3]));
+          const float am = zm * inv_tau;
+          if (!(am + kGumbelMaxF + 1e-4f + 1e-6f * fabsf(am) >= T)) continue;
+          const int v0 = c * 8 + 4 * gq;
+          const U4 w = philox_rk((uint32_t)(v0 >> 2), rid, st.c2, st.c3, K);
+          // With Xm = (max s - T) log2(e), an entry needs u > 1 - e^{s - T} >= 1 - 2^Xm;
+          // u = (m + 1/2) 2^-23 with m = w >> 9, so a word with m below mstar fails for all four.
+          uint32_t mstar = 0;
+          if (T > -INFINITY) {
+            const float thr = (1.0f - ex2(fmaf(zm, cT, -T * kLog2e)) * 1.001f) - 2.4e-7f;
+            mstar = thr > 0.f ? (uint32_t)ceilf(thr * 8388608.f - 0.5f) : 0u;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t wj = word_of(w, j);
+            if ((wj >> 9) < mstar) continue;
+            const float sv = z4[j] * inv_tau;
+            if (!(sv > -INFINITY)) continue;
+            const float u = uniform_f32(wj);
+            if (T > -INFINITY) {  // the entry's own test: u <= 1 - e^{s - T} cannot reach T
+              const float y = ex2((sv - T) * kLog2e) * 1.001f + 1e-30f;
+              if (u < (1.0f - y) - 2.4e-7f) continue;
+            }
+            const float g32 = gumbel_f32(u);
+            const float sc = sv + g32;
+            const float d = score_err(sv, g32);
+            if (!(sc + d >= T)) continue;
+            dropped_hi = fmaxf(dropped_hi, list_insert_col(ls, ldv, li, nthr, k1, sc, d, v0 + j));
+            // lower bound of this thread's (k+1)-th best (-inf until it holds k+1)
+            T = fmaxf(T, ls[(k1 - 1) * nthr] - ldv[(k1 - 1) * nthr]);
+          }
+        }
+      }
+    }
+    atomicMax(&sm.thr, f2ord(T));
+    atomicMax(&sm.dropped, f2ord(dropped_hi));
     __syncthreads();
-    exact_topk_row<TIn>(row, V, k1, inv_tau, tau64, lo_k, st, (uint32_t)r, &sm);
+    // gather the list entries that can still make the top k+1
+    const float Tfin = ord2f(sm.thr);
+    for (int j = 0; j < k1; ++j) {
+      const float cs = ls[j * nthr], cd = ldv[j * nthr];
+      const int ci = li[j * nthr];
+      if (ci != 0x7FFFFFFF && cs + cd >= Tfin) {
+        const int pos = atomicAdd(&sm.ncand, 1);
+        if (pos < kCandCap) {
+          sm.cs[pos] = cs;
+          sm.cd[pos] = cd;
+          sm.ci[pos] = ci;
+        }
+      }
+    }
     __syncthreads();
-  }
-  if (tid < k) {
-    const int v = sm.i64[tid];
-    const bool ok = v != 0x7FFFFFFF && sm.s64[tid] > -INFINITY;
-    idx_out[(int64_t)r * k + tid] = ok ? v : -1;
-    if (score_out) score_out[(int64_t)r * k + tid] = ok ? (float)sm.s64[tid] : NAN;
-    if (logp_out)
-      logp_out[(int64_t)r * k + tid] = ok ? (float)((double)ld_elem<TIn>(row, v) / tau64 - sm.lse) : NAN;
+    if (rowbad) {  // non-finite row
+      if (tid < k) {
+        idx_out[(int64_t)r * k + tid] = -1;
+        if (score_out) score_out[(int64_t)r * k + tid] = NAN;
+        if (logp_out) logp_out[(int64_t)r * k + tid] = NAN;
+      }
+      if (tid == 0) raise_err(dev_err, SD_DEV_NONFINITE);
+      __syncthreads();
+      continue;
+    }
+    const int n = min(sm.ncand, kCandCap);
+    bool need_exact = sm.ncand > kCandCap;
+    // warp 0 extracts the top k+1 (descending, ties to the lower index)
+    if (warp == 0) {
+      bool ambiguous = false;
+      float prev_lo = INFINITY;
+      for (int rnk = 0; rnk < k1; ++rnk) {
+        float bs = -INFINITY, bd = 0.f;
+        int bi = 0x7FFFFFFF, bp = -1;
+        for (int q = lane; q < n; q += 32) {
+          const float sv = sm.cs[q];
+          const int v = sm.ci[q];
+          if (sv > bs || (sv == bs && v < bi)) {
+            bs = sv;
+            bi = v;
+            bd = sm.cd[q];
+            bp = q;
+          }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          const float od = __shfl_xor_sync(0xffffffffu, bd, o);
+          const int op = __shfl_xor_sync(0xffffffffu, bp, o);
+          if (os > bs || (os == bs && oi < bi)) {
+            bs = os;
+            bi = oi;
+            bd = od;
+            bp = op;
+          }
+        }
+        // the order between this rank and the previous one must be settled
+        if (rnk > 0 && bi != 0x7FFFFFFF && !(bs + bd < prev_lo)) ambiguous = true;
+        // nothing evicted from a thread's list may reach the k-th output
+        if (rnk == k - 1 && !(ord2f(sm.dropped) < bs - bd)) ambiguous = true;
+        prev_lo = bs - bd;
+        if (lane == 0) {
+          sm.s64[rnk] = bs;
+          sm.i64[rnk] = bi;
+          if (bp >= 0) sm.cs[bp] = -INFINITY;
+        }
+        __syncwarp();
+      }
+      if (lane == 0 && ambiguous) sm.flag |= 2;
+    }
+    __syncthreads();
+    need_exact = need_exact || (sm.flag & 2);
+    if (need_exact) {
+      // lo bound of the k-th candidate: everything that can reach it is re-scored
+      const float lo_k = (float)sm.s64[k - 1] - 1e-3f - 1e-5f * fabsf((float)sm.s64[k - 1]);
+      __syncthreads();
+      exact_topk_row<TIn>(row, V, k1, inv_tau, tau64, lo_k, st, rid, &sm);
+      __syncthreads();
+    }
+    if (tid < k) {
+      const int v = sm.i64[tid];
+      const bool ok = v != 0x7FFFFFFF && sm.s64[tid] > -INFINITY;
+      idx_out[(int64_t)r * k + tid] = ok ? v : -1;
+      if (score_out) score_out[(int64_t)r * k + tid] = ok ? (float)sm.s64[tid] : NAN;
+      if (logp_out)
+        logp_out[(int64_t)r * k + tid] = ok ? (float)((double)ld_elem<TIn>(row, v) / tau64 - sm.lse) : NAN;
+    }
+    __syncthreads();  // the shared state is reused by the next row
   }
 }
 
@@ -452,24 +628,27 @@ extern "C" sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, in
   const int vec = ((uintptr_t)z % 16 == 0) && ((ld * esize) % 16 == 0);
   const float inv_tau = (float)(1.0 / (double)tau);
   cudaStream_t s = (cudaStream_t)stream;
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SD_ERR_CUDA;
+  }
+  const int grid = std::min(rows, 2 * nsm);  // persistent: two CTAs per SM take the rows in turn
+  // the candidate lists take dynamic shared memory: 3 * L * threads * 4 bytes
+  auto launch = [&](auto kern, int L, const auto* zp) {
+    const int dyn = 3 * L * kTopkThreads * 4;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess)
+      return;
+    kern<<<grid, kTopkThreads, dyn, s>>>(zp, rows, V, ld, k, inv_tau, (double)tau, seed, round, vec,
+                                         idx_out, score_out, logp_out, dev_err);
+  };
   if (dt == SD_BF16) {
-    if (k <= 8)
-      topk_dense_kernel<uint16_t, 9><<<rows, kTopkThreads, 0, s>>>(
-          (const uint16_t*)z, rows, V, ld, k, inv_tau, (double)tau, seed, round, vec, idx_out,
-          score_out, logp_out, dev_err);
-    else
-      topk_dense_kernel<uint16_t, 17><<<rows, kTopkThreads, 0, s>>>(
-          (const uint16_t*)z, rows, V, ld, k, inv_tau, (double)tau, seed, round, vec, idx_out,
-          score_out, logp_out, dev_err);
+    if (k <= 8) launch(topk_dense_kernel<uint16_t, 9>, 9, (const uint16_t*)z);
+    else launch(topk_dense_kernel<uint16_t, 17>, 17, (const uint16_t*)z);
   } else {
-    if (k <= 8)
-      topk_dense_kernel<float, 9><<<rows, kTopkThreads, 0, s>>>(
-          (const float*)z, rows, V, ld, k, inv_tau, (double)tau, seed, round, vec, idx_out,
-          score_out, logp_out, dev_err);
-    else
-      topk_dense_kernel<float, 17><<<rows, kTopkThreads, 0, s>>>(
-          (const float*)z, rows, V, ld, k, inv_tau, (double)tau, seed, round, vec, idx_out,
-          score_out, logp_out, dev_err);
+    if (k <= 8) launch(topk_dense_kernel<float, 9>, 9, (const float*)z);
+    else launch(topk_dense_kernel<float, 17>, 17, (const float*)z);
   }
   return cudaGetLastError() == cudaSuccess ? SD_OK : SD_ERR_CUDA;
 }

@@ -16,7 +16,8 @@ Sources (summaries on gist.science; each function cites its passage):
     (section 2, Methodology); standard SD verification (section 1).
   * STAND (stochastic adaptive n-gram drafting) -- Gumbel-Top-K sampling without
     replacement from stored top-10 (index, probability) rows (Methodology,
-    items 1 and 2).
+    items 1 and 2); stochastic drafting from a distribution rather than its
+    argmax (Methodology, item 1).
 
 Every function's parity status is stated in its docstring.  Functions whose
 randomness is defined by counter-based Philox draws are "pinned by
@@ -25,7 +26,7 @@ definition + statistics": the pages print no worked example with values.
 
 from .philox import (philox4x32_10, uniform_from_bits, gumbel_from_uniform,  # noqa: F401
                      stream_words, STREAM_BONUS, STREAM_ACCEPT, STREAM_RESIDUAL,
-                     STREAM_RESAMPLE, STREAM_TOPK_DENSE, STREAM_TOPK_SPARSE)
+                     STREAM_RESAMPLE, STREAM_TOPK_DENSE, STREAM_TOPK_SPARSE, STREAM_DRAFT)
 from .score import (row_log_softmax, total_variation, smcsd_score,  # noqa: F401
                     DEV_TOKEN_OOB, DEV_NONFINITE, DEV_ZERO_RESIDUAL, DEV_PAGE_OOB,
                     DEV_ANCESTOR_OOB)
@@ -33,3 +34,4 @@ from .resample import smcsd_resample, systematic_ancestors  # noqa: F401
 from .pagetable import kv_pagetable_remap  # noqa: F401
 from .verify import sd_verify_reject, accept_probability, residual_distribution  # noqa: F401
 from .topk import gumbel_topk, gumbel_topk_sparse  # noqa: F401
+from .draft import sd_draft_sample  # noqa: F401

@@ -39,6 +39,7 @@ STREAM_RESIDUAL = 3     # residual-resample Gumbel noise (per vocabulary entry)
 STREAM_RESAMPLE = 4     # systematic-resampling offset u0 (per sequence)
 STREAM_TOPK_DENSE = 5   # dense Gumbel-top-k noise (per vocabulary entry)
 STREAM_TOPK_SPARSE = 6  # sparse Gumbel-top-k noise (per stored entry)
+STREAM_DRAFT = 8        # draft-token Gumbel noise of the draft step (per vocabulary entry)
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1):

@@ -8,6 +8,12 @@ generator, built on the device) and larger than L2, so no flush is needed.
 Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under torchrun;
 each rank runs its own replica of the workload on disjoint sequences (weak
 scaling, no collective on the data path; barrier + max-over-ranks timing).
+
+On one GPU the line also carries `per_config`: the path's other
+configurations (one SMC-SD sequence in fp32, the 64-sequence batch, standard
+verification, dense and sparse Gumbel-top-k) timed on their own with L2
+flushed (and hot where the inputs fit in L2), each with its clocks, its
+algorithmic bytes against the copy peak and its own summary.
 """
 
 import argparse
@@ -375,6 +381,7 @@ def run_ours(args, rank, world, local):
     score_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_pairs)
     score_ms = max_over_ranks(score_ms, world)
     assert int(err.item()) == 0, f"device error word {int(err.item())}"
+    ess_n = (ess / N).cpu().numpy()
 
     rows_per_step = B * N * R
     value = rows_per_step * world * args.steps / (ms * 1e-3)
@@ -399,6 +406,8 @@ def run_ours(args, rank, world, local):
                      "frac_of_nominal_8TBps": achieved / NOMINAL_HBM_GBS},
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
+        "ess_over_N": {"mean": float(ess_n.mean()), "min": float(ess_n.min()),
+                       "max": float(ess_n.max())},
     }
     # End to end through the public API with host buffers (pinned), one replica.
     if args.e2e_steps > 0:
@@ -432,6 +441,8 @@ def run_ours(args, rank, world, local):
                        "unit": "rows/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "steps": args.e2e_steps}
         del h_zT, h_zD
+    if rank == 0 and world == 1 and args.configs:
+        line["per_config"] = per_config(args, hbm_peak, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = oracle_baseline(gen.CONFIGS[WORKLOAD], budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": cores, "kind": "oracle",
@@ -440,105 +451,147 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
-def run_rows(args, workload):
-    """The other rows of the path, each on its own configuration (one GPU, one
-    JSON line each): `verify` = standard SD verification of 128 sequences x
-    (5+1) target / 5 draft rows of V = 32000 bf16 (90 MB, below L2: L2 flushed
-    before every launch); `topk` = Gumbel-top-8 over 4096 x 152064 bf16 rows
-    (1.25 GB) and the sparse variant over 4096 x top-10 stored rows.  Each line
-    has the kernel's event-timed mean, its algorithmic bytes against the
-    measured copy bandwidth, and the oracle timed on a sample of the same rows."""
-    import oracle
+PER_CONFIGS = ("smc_small", "smc_batch", "verify", "topk_dense", "topk_sparse")
+
+
+def per_config(args, hbm_peak, peak_kind):
+    """The path's other configurations, each timed on its own (one GPU): kernel
+    time (mean and median of `args.config_steps` launches, L2 flushed before
+    each by writing 256 MB, plus hot timings where the inputs fit in L2), the
+    algorithmic bytes against the copy-bandwidth peak, the SM clocks sampled
+    while it ran, and the configuration's own summary (ESS of the SMC rounds,
+    the verify accepted-length histogram by draft-noise third)."""
     import resample_online_log_b200 as lib
     from synth import device as sdev
     from synth import gen
 
-    cfg = gen.CONFIGS[workload]
     dev = "cuda"
-    hbm_peak, peak_kind = peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2x L2
     err = torch.zeros((1,), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
+    wanted = [c for c in args.configs.split(",") if c]
+    out = {}
 
-    def timed(call, flush_l2):
-        for i in range(args.warmup):
+    def timed(call, flush_l2, n):
+        for i in range(max(3, args.warmup)):
             call(i)
         torch.cuda.synchronize()
+        clk = ClockSampler(torch.cuda.current_device())
+        clk.start()
+        time.sleep(0.2)
         ts = []
-        for i in range(args.steps):
+        for i in range(n):
             if flush_l2:
                 flush.add_(1)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            call(args.warmup + i)
+            call(100 + i)
             e1.record(stream)
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1))
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        clocks = clk.stop()
+        ms = [a.elapsed_time(b) for a, b in ts]
         assert int(err.item()) == 0, f"device error word {int(err.item())}"
-        return statistics.mean(ts), statistics.median(ts)
+        return statistics.mean(ms), statistics.median(ms), clocks
 
-    def line(name, rows, ms, med, alg_bytes, cpu_rows, cpu_s, sample, extra):
-        achieved = alg_bytes / (ms * 1e-3) / 1e9
-        return {"metric": METRIC, "value": rows / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "ms_median": med,
-                "higher_is_better": True, "data": "synthetic",
-                "config": {"workload": name, **extra},
-                "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                             "frac": achieved / hbm_peak, "peak_kind": peak_kind,
-                             "algorithmic_bytes": alg_bytes},
-                "cpu_baseline": {"value": cpu_rows / cpu_s, "unit": "rows/s", "cores": 1,
-                                 "kind": "oracle", "sample": sample}}
+    def entry(ms, med, alg, units, unit_name, clocks, extra):
+        ach = alg / (ms * 1e-3) / 1e9
+        return {"ms_mean": ms, "ms_median": med, "algorithmic_bytes": alg,
+                "achieved_GBps": ach, "frac": ach / hbm_peak, "peak": hbm_peak,
+                "peak_kind": peak_kind, unit_name: units / (ms * 1e-3), "clocks": clocks, **extra}
 
-    esize = 2 if cfg.dtype == "bf16" else 4
-    out = []
-    if workload == "verify":
-        d = sdev.gen_config_device(cfg)
-        B, K, V = cfg.B, cfg.K, cfg.V
-        acc = torch.empty((B,), dtype=torch.int32, device=dev)
-        toks = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
-        tv = torch.empty((B, K), dtype=torch.float32, device=dev)
-        ms, med = timed(lambda i: lib.sd_verify_reject(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed,
-                                                        i, acc, toks, tv_out=tv, dev_err=err), True)
-        alg = ((2 * K + 1) * V * esize + K * 4 + 4 + (K + 1) * 4 + K * 4) * B
-        h = gen.gen_config_rows(cfg, seqs=list(range(8)))
-        t0 = time.perf_counter()
-        oracle.sd_verify_reject(h["zT"], h["zD"], h["draft"], cfg.tau, cfg.seed, 0)
-        cpu_s = time.perf_counter() - t0
-        out.append(line("verify", B * (K + 1), ms, med, alg, 8 * (K + 1), cpu_s,
-                        "sequences 0-7 of the workload, NumPy fp64, one core",
-                        {"B": B, "K": K, "V": V, "logits": cfg.dtype, "l2": "flushed before each launch"}))
-    else:
-        d = sdev.gen_config_device(cfg)
-        z = d["z"]
-        rows, V, k = z.shape[0], cfg.V, cfg.topk
-        idx = torch.empty((rows, k), dtype=torch.int32, device=dev)
-        sc = torch.empty((rows, k), dtype=torch.float32, device=dev)
-        lp = torch.empty((rows, k), dtype=torch.float32, device=dev)
-        ms, med = timed(lambda i: lib.gumbel_topk(z, k, cfg.tau, cfg.seed, i, idx, score_out=sc,
-                                                  logp_out=lp, dev_err=err), False)
-        alg = rows * (V * esize + k * 12)
-        h = gen.gen_config_rows(cfg, seqs=list(range(16)))
-        t0 = time.perf_counter()
-        oracle.gumbel_topk(h["z"], k, cfg.tau, cfg.seed, 0)
-        cpu_s = time.perf_counter() - t0
-        out.append(line("topk_dense", rows, ms, med, alg, 16, cpu_s,
-                        "rows 0-15 of the workload, NumPy fp64, one core",
-                        {"rows": rows, "V": V, "k": k, "logits": cfg.dtype,
-                         "l2": "inputs (1.2 GB) larger than L2; no flush"}))
-        six, spr = gen.sparse_rows(cfg.seed, rows, cfg.sparse_L, V)
-        ix = torch.from_numpy(six).to(dev)
-        pr = torch.from_numpy(spr.astype(np.float32)).to(dev)
-        ms, med = timed(lambda i: lib.gumbel_topk_sparse(ix, pr, k, cfg.tau, cfg.seed, i, idx,
-                                                         dev_err=err), True)
-        alg = rows * (cfg.sparse_L * 8 + k * 4)
-        t0 = time.perf_counter()
-        oracle.gumbel_topk_sparse(six, spr, k, cfg.tau, cfg.seed, 0)
-        cpu_s = time.perf_counter() - t0
-        out.append(line("topk_sparse", rows, ms, med, alg, rows, cpu_s,
-                        "all rows, NumPy fp64, one core",
-                        {"rows": rows, "L": cfg.sparse_L, "k": k, "l2": "flushed before each launch"}))
-    for o in out:
-        print(json.dumps(o), flush=True)
+    n = args.config_steps
+    for name in wanted:
+        if name in ("smc_small", "smc_batch"):
+            cfg = gen.CONFIGS[name]
+            d = sdev.gen_config_device(cfg)
+            B, N, R, K, V, P = cfg.B, cfg.N, cfg.R, cfg.K, cfg.V, cfg.P
+            pt = torch.from_numpy(gen.page_table(cfg.seed, B, N, P)).to(dev)
+            logw = torch.empty((B, N), dtype=torch.float64, device=dev)
+            bonus = torch.empty((B, N), dtype=torch.int32, device=dev)
+            tv = torch.empty((B, N, R), dtype=torch.float32, device=dev)
+            toks = torch.empty((B, N, R), dtype=torch.int32, device=dev)
+            anc = torch.empty((B, N), dtype=torch.int32, device=dev)
+            ess = torch.empty((B,), dtype=torch.float64, device=dev)
+            pt_out, tok_out = torch.empty_like(pt), torch.empty_like(toks)
+
+            def rnd(i):
+                lib.smcsd_score(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed, i, logw, bonus,
+                                tv_out=tv, tokens_out=toks, dev_err=err)
+                lib.smcsd_resample(logw, cfg.seed, i, anc, ess_out=ess, dev_err=err)
+                lib.kv_pagetable_remap(pt, anc, pt_out, tok_in=toks, tok_out=tok_out, dev_err=err)
+            esize = 2 if cfg.dtype == "bf16" else 4
+            alg = (2 * B * N * R * V * esize + B * N * K * 4 + B * N * 12 + B * N * R * 8
+                   + 2 * B * N * P * 4 + 2 * B * N * R * 4)
+            ms, med, clocks = timed(rnd, True, n)
+            ess_n = (ess / N).cpu().numpy()
+            extra = {"config": {"B": B, "N": N, "K": K, "V": V, "logits": cfg.dtype, "tau": cfg.tau,
+                                "step": "score -> resample -> page-table remap", "l2": "flushed"},
+                     "ess_over_N": {"mean": float(ess_n.mean()), "min": float(ess_n.min()),
+                                    "max": float(ess_n.max())}}
+            if 2 * B * N * R * V * esize < (60 << 20):  # fits in L2: the hot figure too
+                hms, hmed, _ = timed(rnd, False, n)
+                extra["hot_ms_mean"], extra["hot_ms_median"] = hms, hmed
+            out[name] = entry(ms, med, alg, B * N * R, "rows_per_s", clocks, extra)
+            del d
+        elif name == "verify":
+            cfg = gen.CONFIGS["verify"]
+            d = sdev.gen_config_device(cfg)
+            B, K, V = cfg.B, cfg.K, cfg.V
+            acc = torch.empty((B,), dtype=torch.int32, device=dev)
+            toks = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+            tv = torch.empty((B, K), dtype=torch.float32, device=dev)
+
+            def ver(i):
+                lib.sd_verify_reject(d["zT"], d["zD"], d["draft"], cfg.tau, cfg.seed, i, acc, toks,
+                                     tv_out=tv, dev_err=err)
+            alg = ((2 * K + 1) * V * 2 + K * 4 + 4 + (K + 1) * 4 + K * 4) * B
+            ms, med, clocks = timed(ver, True, n)
+            hms, hmed, _ = timed(ver, False, n)
+            a = acc.cpu().numpy()
+            thirds = [(0, 43), (43, 86), (86, 128)]
+            hist = {f"sigma_{sd}": np.bincount(a[lo:hi], minlength=K + 1).tolist()
+                    for (lo, hi), sd in zip(thirds, cfg.sigma_d)}
+            out[name] = entry(ms, med, alg, B * (K + 1), "target_rows_per_s", clocks,
+                              {"config": {"B": B, "K": K, "V": V, "logits": cfg.dtype, "tau": cfg.tau,
+                                          "l2": "flushed; hot_* without the flush"},
+                               "hot_ms_mean": hms, "hot_ms_median": hmed,
+                               "accepted_len_hist_by_draft_noise": hist})
+            del d
+        elif name in ("topk_dense", "topk_sparse"):
+            cfg = gen.CONFIGS["topk"]
+            rows, V, k = cfg.B, cfg.V, cfg.topk
+            idx = torch.empty((rows, k), dtype=torch.int32, device=dev)
+            if name == "topk_dense":
+                z = sdev.gen_config_device(cfg)["z"]
+                sc = torch.empty((rows, k), dtype=torch.float32, device=dev)
+                lp = torch.empty((rows, k), dtype=torch.float32, device=dev)
+
+                def tk(i):
+                    lib.gumbel_topk(z, k, cfg.tau, cfg.seed, i, idx, score_out=sc, logp_out=lp,
+                                    dev_err=err)
+                alg = rows * (V * 2 + k * 12)
+                ms, med, clocks = timed(tk, True, n)
+                out[name] = entry(ms, med, alg, rows, "rows_per_s", clocks,
+                                  {"config": {"rows": rows, "V": V, "k": k, "logits": cfg.dtype,
+                                              "tau": cfg.tau, "l2": "flushed"}})
+                del z
+            else:
+                six, spr = gen.sparse_rows(cfg.seed, rows, cfg.sparse_L, V)
+                ix = torch.from_numpy(six).to(dev)
+                pr = torch.from_numpy(spr.astype(np.float32)).to(dev)
+
+                def tks(i):
+                    lib.gumbel_topk_sparse(ix, pr, k, cfg.tau, cfg.seed, i, idx, dev_err=err)
+                alg = rows * (cfg.sparse_L * 8 + k * 4)
+                ms, med, clocks = timed(tks, True, n)
+                hms, hmed, _ = timed(tks, False, n)
+                out[name] = entry(ms, med, alg, rows, "rows_per_s", clocks,
+                                  {"config": {"rows": rows, "L": cfg.sparse_L, "k": k, "tau": cfg.tau,
+                                              "l2": "flushed; hot_* without the flush"},
+                                   "hot_ms_mean": hms, "hot_ms_median": hmed})
+        torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -552,11 +605,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sequences", type=int, default=0,
                     help="run B sequences of the workload instead of all 256 (profiling)")
-    ap.add_argument("--workload", choices=[WORKLOAD, "verify", "topk"], default=WORKLOAD,
-                    help="verify / topk: the path's other rows, timed on their own configs (1 GPU)")
+    ap.add_argument("--configs", default=",".join(PER_CONFIGS),
+                    help="the other configurations timed into per_config (empty: none)")
+    ap.add_argument("--config-steps", type=int, default=20)
+    ap.add_argument("--per-config-only", action="store_true",
+                    help="print only the per_config object (one GPU)")
     args = ap.parse_args()
-    if args.workload != WORKLOAD:
-        run_rows(args, args.workload)
+    if args.per_config_only:
+        hbm_peak, peak_kind = peaks()
+        print(json.dumps({"per_config": per_config(args, hbm_peak, peak_kind)}), flush=True)
         return
     rank, world, local = dist_init()
     try:

@@ -80,6 +80,7 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_STREAM_RESAMPLE 4u
 #define SD_STREAM_TOPK_DENSE 5u
 #define SD_STREAM_TOPK_SPARSE 6u
+#define SD_STREAM_DRAFT 8u
 
 /*
  * smcsd_score -- scoring step of one SMC-SD round ([SMC-SD] section 2, scoring
@@ -213,6 +214,31 @@ SMCSD_API sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, int
 SMCSD_API sd_status gumbel_topk_sparse(const int32_t* idx, const float* prob, int rows, int L, int k,
                              float tau, uint64_t seed, uint64_t round, int32_t* idx_out,
                              uint32_t* dev_err, void* stream);
+
+/*
+ * sd_draft_sample -- the draft step's sampling: one token per draft row drawn
+ * from the drafter's own distribution ([SMC-SD] section 2: the draft model
+ * extends each particle by K tokens, one position at a time; [STAND]
+ * Methodology item 1: stochastic drafting samples the distribution instead of
+ * taking its argmax).  Gumbel-max, exact:
+ *   tokens[r] = argmax_v (zD[r, v] / tau + g_v), g from stream 8 with row id
+ *               row0 + r, ties to the lower v;
+ *   logq[r]   = zD[r, tokens[r]] / tau - logsumexp_v(zD[r, v] / tau),
+ * the log q_D(x) an SMC-SD importance weight uses.  One call per draft
+ * position: rows are all particles of all sequences at that position.
+ * zD          device [rows, V] at row stride ld, dtype dt.
+ * row0        row id of the first row (the noise of row r uses row0 + r;
+ *             row0 + rows <= 2^32).
+ * tokens_out  device int32 [rows]                           (required)
+ * logq_out    device fp32 [rows]                            (or NULL)
+ * Requirements: rows >= 0, V >= 1, ld >= V, tau > 0 finite.
+ * Faults: rows with NaN / +inf or all -inf -> SD_DEV_NONFINITE, token -1,
+ *   logq NaN.
+ */
+SMCSD_API sd_status sd_draft_sample(const void* zD, sd_dtype dt, int rows, int V, int64_t ld,
+                                    float tau, uint64_t seed, uint64_t round, uint32_t row0,
+                                    int32_t* tokens_out, float* logq_out, uint32_t* dev_err,
+                                    void* stream);
 
 /* Human-readable name of a status code (static storage). */
 SMCSD_API const char* sd_status_string(sd_status s);

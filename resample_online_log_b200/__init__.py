@@ -22,7 +22,8 @@ DEV_TOKEN_OOB, DEV_NONFINITE, DEV_ZERO_RESIDUAL = 1, 2, 4
 DEV_PAGE_OOB, DEV_ANCESTOR_OOB, DEV_TIMEOUT = 8, 16, 32
 
 EXPORTS = ("smcsd_score", "smcsd_resample", "kv_pagetable_remap", "sd_verify_reject",
-           "gumbel_topk", "gumbel_topk_sparse", "sd_status_string", "sd_version")
+           "gumbel_topk", "gumbel_topk_sparse", "sd_draft_sample", "sd_status_string",
+           "sd_version")
 
 _lib = None
 
@@ -52,7 +53,9 @@ def load():
                                    vp, vp]
     L.gumbel_topk.argtypes = [vp, i32, i32, i32, i64, i32, f32, u64, u64, vp, vp, vp, vp, vp]
     L.gumbel_topk_sparse.argtypes = [vp, vp, i32, i32, i32, f32, u64, u64, vp, vp, vp]
-    for name in EXPORTS[:6]:
+    L.sd_draft_sample.argtypes = [vp, i32, i32, i32, i64, f32, u64, u64, ctypes.c_uint32, vp, vp,
+                                  vp, vp]
+    for name in EXPORTS[:7]:
         getattr(L, name).restype = ctypes.c_int
     L.sd_status_string.argtypes = [ctypes.c_int]
     L.sd_status_string.restype = ctypes.c_char_p
@@ -226,3 +229,17 @@ def gumbel_topk_sparse(idx, prob, k, tau, seed, round, idx_out, dev_err=None, st
     st = load().gumbel_topk_sparse(_p(idx), _p(prob), rows, L, int(k), float(tau), int(seed),
                                    int(round), _p(idx_out), _p(dev_err), _stream(stream))
     _check("gumbel_topk_sparse", st)
+
+
+def sd_draft_sample(zD, tau, seed, round, tokens_out, logq_out=None, row0=0, dev_err=None,
+                    stream=None):
+    """zD: [rows, V] draft logits (bf16 or fp32); tokens_out int32 [rows]."""
+    rows = zD.shape[0]
+    V, ld = _rows_view(zD, (rows,))
+    _want(tokens_out, torch.int32, (rows,), "tokens_out")
+    _want(logq_out, torch.float32, (rows,), "logq_out")
+    _check_err(dev_err)
+    st = load().sd_draft_sample(_p(zD), _dtype(zD), rows, V, ld, float(tau), int(seed), int(round),
+                                int(row0), _p(tokens_out), _p(logq_out), _p(dev_err),
+                                _stream(stream))
+    _check("sd_draft_sample", st)

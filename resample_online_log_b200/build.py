@@ -8,6 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = ["abi.cu", "smc.cu", "verify.cu", "resample.cu", "pagetable.cu", "topk.cu"]
 LIB = os.path.join(HERE, "libsmcsd.so")
+TESTING_LIB = os.path.join(HERE, "libsmcsd_testing.so")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 
@@ -36,6 +37,13 @@ def build(verbose=False, jobs=None):
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)
+    # Test-only library: the device generator on chosen counters (tests pin it).
+    tobj = os.path.join(objdir, "testing.o")
+    subprocess.check_call(["nvcc", *FLAGS, "-I", inc, "-c", os.path.join(csrc, "testing.cu"),
+                           "-o", tobj])
+    subprocess.check_call(["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
+                           "--cudart", "static", "-Xlinker", "--exclude-libs,ALL", "-o",
+                           TESTING_LIB, tobj])
     return LIB
 
 

@@ -310,14 +310,14 @@ __device__ __noinline__ float cta_kth_largest(float v, int k, float* buf /* [nwa
 template <typename TIn, int L>
 __global__ void __launch_bounds__(kTopkThreads, 2) topk_dense_kernel(
     const TIn* __restrict__ z, int rows, int V, int64_t ld, int k, float inv_tau, double tau64,
-    uint64_t seed, uint64_t round, int vec, int32_t* __restrict__ idx_out, float* score_out,
-    float* logp_out, uint32_t* dev_err) {
+    uint64_t seed, uint64_t round, uint32_t tag, uint32_t row0, int vec,
+    int32_t* __restrict__ idx_out, float* score_out, float* logp_out, uint32_t* dev_err) {
   __shared__ TopkSmem sm;
   __shared__ float kbuf[(kTopkThreads / 32) * kTopkMax];
   extern __shared__ float lists[];  // [3][L][blockDim.x]: scores, error bounds, indices
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x;
   const int k1 = k + 1;
-  const Stream st(seed, round, SD_STREAM_TOPK_DENSE);
+  const Stream st(seed, round, tag);
   const PhiloxKeys K = philox_keys(seed);
   const float cT = kLog2e * inv_tau;  // log2(e) / tau
   const int nchunks = (V + 7) / 8;
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_dense_kernel(
 
   for (int r = blockIdx.x; r < rows; r += gridDim.x) {
     const TIn* row = z + (int64_t)r * ld;
-    const uint32_t rid = (uint32_t)r;
+    const uint32_t rid = row0 + (uint32_t)r;
     if (tid == 0) {
       sm.thr = f2ord(-INFINITY);
       sm.dropped = f2ord(-INFINITY);
@@ -614,20 +614,17 @@ __global__ void topk_sparse_kernel(const int32_t* __restrict__ idx, const float*
 
 using namespace smcsd;
 
-extern "C" sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, int64_t ld, int k,
-                                 float tau, uint64_t seed, uint64_t round, int32_t* idx_out,
-                                 float* score_out, float* logp_out, uint32_t* dev_err,
-                                 void* stream) {
-  if (rows < 0 || V < 1 || ld < V || k < 1 || k > kTopkMax || k > V ||
-      !(tau > 0.f && tau < INFINITY))
-    return SD_ERR_INVALID_ARG;
-  if (dt != SD_F32 && dt != SD_BF16) return SD_ERR_INVALID_ARG;
-  if (rows == 0) return SD_OK;
-  if (!z || !idx_out) return SD_ERR_INVALID_ARG;
+namespace smcsd {
+
+// Launches the dense kernel: k ranks of rows [rows, V] with noise stream `tag`
+// and row ids row0, row0 + 1, ...
+static sd_status launch_topk_dense(const void* z, sd_dtype dt, int rows, int V, int64_t ld, int k,
+                                   float tau, uint64_t seed, uint64_t round, uint32_t tag,
+                                   uint32_t row0, int32_t* idx_out, float* score_out,
+                                   float* logp_out, uint32_t* dev_err, cudaStream_t s) {
   const int esize = dt == SD_BF16 ? 2 : 4;
   const int vec = ((uintptr_t)z % 16 == 0) && ((ld * esize) % 16 == 0);
   const float inv_tau = (float)(1.0 / (double)tau);
-  cudaStream_t s = (cudaStream_t)stream;
   int dev = 0, nsm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
@@ -640,8 +637,8 @@ extern "C" sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, in
     const int dyn = 3 * L * kTopkThreads * 4;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn) != cudaSuccess)
       return;
-    kern<<<grid, kTopkThreads, dyn, s>>>(zp, rows, V, ld, k, inv_tau, (double)tau, seed, round, vec,
-                                         idx_out, score_out, logp_out, dev_err);
+    kern<<<grid, kTopkThreads, dyn, s>>>(zp, rows, V, ld, k, inv_tau, (double)tau, seed, round, tag,
+                                         row0, vec, idx_out, score_out, logp_out, dev_err);
   };
   if (dt == SD_BF16) {
     if (k <= 8) launch(topk_dense_kernel<uint16_t, 9>, 9, (const uint16_t*)z);
@@ -651,6 +648,37 @@ extern "C" sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, in
     else launch(topk_dense_kernel<float, 17>, 17, (const float*)z);
   }
   return cudaGetLastError() == cudaSuccess ? SD_OK : SD_ERR_CUDA;
+}
+
+}  // namespace smcsd
+
+extern "C" sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, int64_t ld, int k,
+                                 float tau, uint64_t seed, uint64_t round, int32_t* idx_out,
+                                 float* score_out, float* logp_out, uint32_t* dev_err,
+                                 void* stream) {
+  if (rows < 0 || V < 1 || ld < V || k < 1 || k > kTopkMax || k > V ||
+      !(tau > 0.f && tau < INFINITY))
+    return SD_ERR_INVALID_ARG;
+  if (dt != SD_F32 && dt != SD_BF16) return SD_ERR_INVALID_ARG;
+  if (rows == 0) return SD_OK;
+  if (!z || !idx_out) return SD_ERR_INVALID_ARG;
+  return launch_topk_dense(z, dt, rows, V, ld, k, tau, seed, round, SD_STREAM_TOPK_DENSE, 0u,
+                           idx_out, score_out, logp_out, dev_err, (cudaStream_t)stream);
+}
+
+// Draft step: one token per row from q_D = softmax(zD / tau) by Gumbel-max, which
+// is Gumbel-top-1: the dense kernel with k = 1 on its own noise stream.
+extern "C" sd_status sd_draft_sample(const void* zD, sd_dtype dt, int rows, int V, int64_t ld,
+                                     float tau, uint64_t seed, uint64_t round, uint32_t row0,
+                                     int32_t* tokens_out, float* logq_out, uint32_t* dev_err,
+                                     void* stream) {
+  if (rows < 0 || V < 1 || ld < V || !(tau > 0.f && tau < INFINITY)) return SD_ERR_INVALID_ARG;
+  if (dt != SD_F32 && dt != SD_BF16) return SD_ERR_INVALID_ARG;
+  if (rows == 0) return SD_OK;
+  if (!zD || !tokens_out) return SD_ERR_INVALID_ARG;
+  if ((uint64_t)row0 + (uint64_t)rows > 0x100000000ull) return SD_ERR_INVALID_ARG;
+  return launch_topk_dense(zD, dt, rows, V, ld, 1, tau, seed, round, SD_STREAM_DRAFT, row0,
+                           tokens_out, nullptr, logq_out, dev_err, (cudaStream_t)stream);
 }
 
 extern "C" sd_status gumbel_topk_sparse(const int32_t* idx, const float* prob, int rows, int L,

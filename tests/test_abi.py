@@ -71,6 +71,12 @@ def test_host_argument_checks_need_no_gpu():
                          None) == lib.SD_ERR_INVALID_ARG            # k > V
     assert L.gumbel_topk_sparse(vp(1), vp(1), 1, 10, 11, 1.0, 0, 0, vp(1), None,
                                 None) == lib.SD_ERR_INVALID_ARG     # k > L
+    assert L.sd_draft_sample(vp(1), 1, 4, 10, 10, 0.0, 0, 0, 0, vp(1), None, None,
+                             None) == lib.SD_ERR_INVALID_ARG        # tau <= 0
+    assert L.sd_draft_sample(vp(1), 1, 4, 10, 10, 1.0, 0, 0, 0xFFFFFFFE, vp(1), None, None,
+                             None) == lib.SD_ERR_INVALID_ARG        # row ids past 2^32
+    assert L.sd_draft_sample(None, 1, 0, 10, 10, 1.0, 0, 0, 0, None, None, None,
+                             None) == lib.SD_OK                     # no rows: nothing to do
 
 
 def test_product_path_has_no_oracle_dependency():
@@ -93,3 +99,16 @@ def test_binding_rejects_a_bad_error_word():
     with pytest.raises(ValueError):
         lib._check_err(torch.zeros((1,), dtype=torch.float32))
     lib._check_err(None)
+
+
+def test_testing_library_exports_its_probes():
+    """libsmcsd_testing.so (built beside the library, used by the GPU pins only)
+    exports the device-generator probes; libsmcsd.so does not."""
+    tl = os.path.join(os.path.dirname(lib.LIB_PATH), "libsmcsd_testing.so")
+    assert os.path.exists(tl), "build the libraries first (__graft_entry__.build())"
+    names = subprocess.run(["nm", "-D", "--defined-only", tl], capture_output=True, text=True,
+                           check=True).stdout
+    assert "smcsd_testing_philox" in names and "smcsd_testing_stream" in names
+    main = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                          text=True, check=True).stdout
+    assert "smcsd_testing" not in main

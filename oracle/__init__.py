@@ -30,7 +30,7 @@ from .philox import (philox4x32_10, uniform_from_bits, gumbel_from_uniform,  # n
 from .score import (row_log_softmax, total_variation, smcsd_score,  # noqa: F401
                     DEV_TOKEN_OOB, DEV_NONFINITE, DEV_ZERO_RESIDUAL, DEV_PAGE_OOB,
                     DEV_ANCESTOR_OOB)
-from .resample import smcsd_resample, systematic_ancestors  # noqa: F401
+from .resample import smcsd_resample, smcsd_resample_adaptive, systematic_ancestors  # noqa: F401
 from .pagetable import kv_pagetable_remap  # noqa: F401
 from .verify import sd_verify_reject, accept_probability, residual_distribution  # noqa: F401
 from .topk import gumbel_topk, gumbel_topk_sparse  # noqa: F401

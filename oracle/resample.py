@@ -76,3 +76,41 @@ def smcsd_resample(logw, seed, rnd, b0=0):
         ess[b] = 1.0 / np.sum(W[b] ** 2)
         anc[b], margin[b] = systematic_ancestors(W[b], resample_offset(seed, rnd, b0 + b))
     return dict(W=W, ess=ess, ancestors=anc, margin=margin, err=err)
+
+
+def smcsd_resample_adaptive(logw, ess_frac, seed, rnd, b0=0):
+    """Adaptive resampling: a sequence is resampled only when its ESS falls below
+    ess_frac * N.
+
+    "Faster LLM Inference via Sequential Monte Carlo", sections 2 (resampling
+    step) and 5 (extensions): resampling every round is the page's scheme; the
+    usual SMC refinement resamples only when the weights have degenerated, the
+    effective sample size being the standard trigger.  Reading: for each
+    sequence compute W and ESS as smcsd_resample does;
+        resampled = ESS < ess_frac * N        (strict; ess_frac > 1: always)
+        ancestors = systematic(W, u0) if resampled else the identity
+        logw_next = 0 if resampled else logw  (the weights carry to the next round)
+    A sequence with NaN / +inf weights, or all -inf, is not resampled: identity
+    ancestors, NaN W and ESS, logw_next = logw, the non-finite error bit.
+
+    Returns dict(W, ess, ancestors, resampled [B] int, logw_next [B, N], margin, err).
+    Parity status: pinned by the never / always limits, exact ESS at the
+    threshold, and the reward-weighted closed form (tests/test_oracle_resample.py).
+    """
+    logw = np.asarray(logw, dtype=np.float64)
+    B, N = logw.shape
+    r = smcsd_resample(logw, seed, rnd, b0=b0)
+    resampled = np.zeros(B, dtype=np.int64)
+    anc = np.tile(np.arange(N, dtype=np.int64), (B, 1))
+    margin = np.full((B, N), np.inf)
+    logw_next = logw.copy()
+    for b in range(B):
+        if np.isnan(r["ess"][b]):
+            continue
+        if r["ess"][b] < ess_frac * N:
+            resampled[b] = 1
+            anc[b] = r["ancestors"][b]
+            margin[b] = r["margin"][b]
+            logw_next[b] = 0.0
+    return dict(W=r["W"], ess=r["ess"], ancestors=anc, resampled=resampled, logw_next=logw_next,
+                margin=margin, err=r["err"])

@@ -86,7 +86,7 @@ def bonus_noise(seed, rnd, row_id, V):
     return gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_BONUS, row_id, V)))
 
 
-def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None, b0=0):
+def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None, b0=0, log_potential=None):
     """Score one SMC-SD round for B sequences x N particles x (K+1) positions.
 
     zT, zD: [B, N, K+1, V] target / draft logits (any float dtype; widened to fp64).
@@ -94,6 +94,12 @@ def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None, b0=0):
     logw_prev: optional [B, N] fp64 log-weights carried from the last round.
     b0: global index of the first sequence when these B sequences are a sample
         of a larger batch (Philox row ids use the global particle index).
+    log_potential: optional [B, N] fp64 extra log-potential per particle
+        ("Faster LLM Inference via Sequential Monte Carlo", section 5: the
+        method extends to constrained and reward-weighted decoding).  Reading:
+        the target of the round becomes p_T(x) phi(x) for a caller-given
+        potential phi (a reward, or 0 / 1 for a constraint), so the importance
+        weight gains the factor phi: logw += log phi (-inf drops the particle).
 
     Returns a dict with
       lse    [B, N, K+1, 2]  (lse of target row, lse of draft row)
@@ -129,6 +135,8 @@ def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None, b0=0):
             lse[b, n, :, 1] = lse_d
             tv[b, n] = total_variation(a, lse_t, d, lse_d)
             acc = 0.0 if logw_prev is None else float(logw_prev[b, n])
+            if log_potential is not None:
+                acc += float(log_potential[b, n])
             for k in range(K):
                 x = int(draft_tokens[b, n, k])
                 if 0 <= x < V:

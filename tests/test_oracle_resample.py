@@ -81,3 +81,56 @@ def test_offset_stream_and_nonfinite():
     assert out["err"] & oracle.DEV_NONFINITE
     assert np.all(np.isnan(out["W"][0])) and np.array_equal(out["ancestors"][0], [0, 1])
     assert np.isfinite(out["W"][1]).all()
+
+
+def test_adaptive_limits():
+    """ess_frac = 0: never resampled (identity, weights carried); ess_frac > 1:
+    always, and then exactly smcsd_resample with log-weights reset to 0."""
+    rng = np.random.default_rng(7)
+    lw = rng.standard_normal((5, 16)) * 2
+    never = oracle.smcsd_resample_adaptive(lw, 0.0, 3, 1)
+    assert (never["resampled"] == 0).all()
+    assert np.array_equal(never["ancestors"], np.tile(np.arange(16), (5, 1)))
+    assert np.array_equal(never["logw_next"], lw)
+    always = oracle.smcsd_resample_adaptive(lw, 2.0, 3, 1)
+    ref = oracle.smcsd_resample(lw, 3, 1)
+    assert (always["resampled"] == 1).all()
+    assert np.array_equal(always["ancestors"], ref["ancestors"])
+    assert (always["logw_next"] == 0).all()
+    assert np.allclose(always["ess"], ref["ess"], rtol=0, atol=0)
+
+
+def test_adaptive_threshold_is_exact_at_known_ess():
+    """k equal weights and N - k zero weights (-inf) give ESS = k exactly: the
+    sequence is resampled iff k < ess_frac * N (strict)."""
+    N = 8
+    lw = np.full((N, N), -np.inf)
+    for k in range(1, N + 1):
+        lw[k - 1, :k] = 0.3
+    out = oracle.smcsd_resample_adaptive(lw, 0.5, 1, 0)  # threshold ESS < 4
+    assert np.allclose(out["ess"], np.arange(1, N + 1), atol=1e-12)
+    assert list(out["resampled"]) == [1, 1, 1, 0, 0, 0, 0, 0]
+    # resampled sequences never pick a zero-weight particle
+    for k in range(1, 4):
+        assert out["ancestors"][k - 1].max() < k
+
+
+def test_reward_weighted_target_closed_form():
+    """With identical target and draft rows the draft terms cancel (logw = 0), so
+    a log-potential phi makes W = softmax(phi) exactly; phi = -inf drops a particle."""
+    rng = np.random.default_rng(8)
+    B, N, K, V = 2, 6, 2, 50
+    zT = rng.standard_normal((B, N, K + 1, V))
+    x = rng.integers(0, V, (B, N, K))
+    phi = rng.standard_normal((B, N))
+    phi[1, 2] = -np.inf
+    o = oracle.smcsd_score(zT, zT.copy(), x, 1.0, 0, 0, log_potential=phi)
+    assert np.array_equal(o["logw"], phi)
+    r = oracle.smcsd_resample(o["logw"], 0, 0)
+    W = np.exp(phi - phi.max(axis=1, keepdims=True))
+    W /= W.sum(axis=1, keepdims=True)
+    assert np.allclose(r["W"], W, atol=1e-15)
+    assert 2 not in r["ancestors"][1]
+    # the potential enters like a carried weight
+    o2 = oracle.smcsd_score(zT, zT.copy(), x, 1.0, 0, 0, logw_prev=np.where(np.isinf(phi), -np.inf, phi))
+    assert np.array_equal(o2["logw"], o["logw"])

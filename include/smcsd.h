@@ -90,7 +90,8 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
  * q = softmax(zD/tau) per row (the same tau divides both):
  *   lse       of every target and draft row;
  *   log-probs lp = log p(x_{k+1}), lq = log q(x_{k+1}) at rows k < K;
- *   logw[b,n] = logw_prev[b,n] + sum_{k<K} (lp - lq)     (importance weight);
+ *   logw[b,n] = logw_prev[b,n] + phi[b,n] + sum_{k<K} (lp - lq)
+ *                                                         (importance weight);
  *   tv[b,n,k] = 1/2 sum_v |p_v - q_v| at all K+1 rows    (block divergence);
  *   bonus[b,n] = argmax_v (zT[b,n,K,v]/tau + g_v), g from stream 1 with row
  *                id b*N+n, ties to the lower v           (bonus token).
@@ -100,6 +101,11 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
  * draft_tokens  device int32 [B, N, K]: token x_{k+1} scored at row k.
  * tau           > 0, finite.
  * logw_prev     device fp64 [B, N] or NULL (NULL = 0, i.e. after resampling).
+ * log_potential device fp64 [B, N] or NULL (NULL = 0): phi, a per-particle
+ *               log-potential multiplied into the target (reward-weighted or
+ *               constrained targets, [SMC-SD] section 5: the target becomes
+ *               p(x) * exp(phi(x)), so the importance weight gains phi).
+ *               -inf marks a particle the constraint rules out (weight 0).
  * logw_out      device fp64 [B, N]                       (required)
  * bonus_out     device int32 [B, N]                      (required)
  * tv_out        device fp32 [B, N, K+1]                  (or NULL)
@@ -114,9 +120,9 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
  */
 SMCSD_API sd_status smcsd_score(const void* zT, const void* zD, sd_dtype dt, int B, int N, int K, int V,
                       int64_t ld, const int32_t* draft_tokens, float tau, uint64_t seed,
-                      uint64_t round, const double* logw_prev, double* logw_out,
-                      int32_t* bonus_out, float* tv_out, int32_t* tokens_out, double* lse_out,
-                      double* lp_out, uint32_t* dev_err, void* stream);
+                      uint64_t round, const double* logw_prev, const double* log_potential,
+                      double* logw_out, int32_t* bonus_out, float* tv_out, int32_t* tokens_out,
+                      double* lse_out, double* lp_out, uint32_t* dev_err, void* stream);
 
 /*
  * smcsd_resample -- weight normalisation, ESS and systematic resampling
@@ -135,6 +141,31 @@ SMCSD_API sd_status smcsd_score(const void* zT, const void* zD, sd_dtype dt, int
 SMCSD_API sd_status smcsd_resample(const double* logw, int B, int N, uint64_t seed, uint64_t round,
                          double* w_out, double* ess_out, int32_t* ancestors_out,
                          uint32_t* dev_err, void* stream);
+
+/*
+ * smcsd_resample_adaptive -- smcsd_resample run only where the weights have
+ * degenerated: sequence b is resampled iff ess[b] < ess_frac * N (strict).
+ * This is the ESS-triggered resampling of standard SMC, which [SMC-SD]
+ * section 5 lists among the extensions of the every-round scheme of
+ * section 2.  A sequence that is not resampled keeps its particles
+ * (identity ancestors) and carries its log-weights into the next round.
+ *   W, ess         as smcsd_resample (always written when requested);
+ *   anc[b,:]       systematic ancestors if resampled, else 0..N-1;
+ *   resampled[b]   1 if resampled, else 0;
+ *   logw_next[b,:] 0 if resampled, else logw[b,:] (the next round's
+ *                  logw_prev for smcsd_score).
+ * ess_frac       >= 0 and not NaN; +inf resamples every sequence (= smcsd_resample),
+ *                0 none.  Typical: 0.5.
+ * resampled_out  device int32 [B] or NULL; logw_next device fp64 [B, N] or
+ *                NULL (may equal logw: each entry is read before it is written
+ *                by the same thread).
+ * Requirements and faults: as smcsd_resample; a faulty sequence is never
+ *   resampled (resampled 0, logw_next = logw).
+ */
+SMCSD_API sd_status smcsd_resample_adaptive(const double* logw, int B, int N, double ess_frac,
+                                  uint64_t seed, uint64_t round, double* w_out, double* ess_out,
+                                  int32_t* ancestors_out, int32_t* resampled_out,
+                                  double* logw_next, uint32_t* dev_err, void* stream);
 
 /*
  * kv_pagetable_remap -- KV cache update after resampling by page-pointer /

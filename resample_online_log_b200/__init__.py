@@ -21,9 +21,9 @@ SD_F32, SD_BF16 = 0, 1
 DEV_TOKEN_OOB, DEV_NONFINITE, DEV_ZERO_RESIDUAL = 1, 2, 4
 DEV_PAGE_OOB, DEV_ANCESTOR_OOB, DEV_TIMEOUT = 8, 16, 32
 
-EXPORTS = ("smcsd_score", "smcsd_resample", "kv_pagetable_remap", "sd_verify_reject",
-           "gumbel_topk", "gumbel_topk_sparse", "sd_draft_sample", "sd_status_string",
-           "sd_version")
+EXPORTS = ("smcsd_score", "smcsd_resample", "smcsd_resample_adaptive", "kv_pagetable_remap",
+           "sd_verify_reject", "gumbel_topk", "gumbel_topk_sparse", "sd_draft_sample",
+           "sd_status_string", "sd_version")
 
 _lib = None
 
@@ -45,9 +45,11 @@ def load():
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, i64, u64, f32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
                               ctypes.c_float)
+    f64 = ctypes.c_double
     L.smcsd_score.argtypes = [vp, vp, i32, i32, i32, i32, i32, i64, vp, f32, u64, u64, vp, vp, vp,
-                              vp, vp, vp, vp, vp, vp]
+                              vp, vp, vp, vp, vp, vp, vp]
     L.smcsd_resample.argtypes = [vp, i32, i32, u64, u64, vp, vp, vp, vp, vp]
+    L.smcsd_resample_adaptive.argtypes = [vp, i32, i32, f64, u64, u64, vp, vp, vp, vp, vp, vp, vp]
     L.kv_pagetable_remap.argtypes = [vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, i32, vp, vp]
     L.sd_verify_reject.argtypes = [vp, vp, i32, i32, i32, i32, i64, vp, f32, u64, u64, vp, vp, vp,
                                    vp, vp]
@@ -55,7 +57,7 @@ def load():
     L.gumbel_topk_sparse.argtypes = [vp, vp, i32, i32, i32, f32, u64, u64, vp, vp, vp]
     L.sd_draft_sample.argtypes = [vp, i32, i32, i32, i64, f32, u64, u64, ctypes.c_uint32, vp, vp,
                                   vp, vp]
-    for name in EXPORTS[:7]:
+    for name in EXPORTS[:8]:
         getattr(L, name).restype = ctypes.c_int
     L.sd_status_string.argtypes = [ctypes.c_int]
     L.sd_status_string.restype = ctypes.c_char_p
@@ -129,8 +131,9 @@ def _want(t, dtype, shape, name):
 
 def smcsd_score(zT, zD, draft_tokens, tau, seed, round, logw_out, bonus_out, logw_prev=None,
                 tv_out=None, tokens_out=None, lse_out=None, lp_out=None, dev_err=None,
-                stream=None):
-    """zT, zD: [B, N, K+1, V] (bf16 or fp32); draft_tokens int32 [B, N, K]."""
+                stream=None, log_potential=None):
+    """zT, zD: [B, N, K+1, V] (bf16 or fp32); draft_tokens int32 [B, N, K];
+    log_potential: fp64 [B, N] added to every particle's log-weight (or None)."""
     B, N, R = zT.shape[:3]
     K = R - 1
     V, ld = _rows_view(zT, (B, N, R))
@@ -141,13 +144,15 @@ def smcsd_score(zT, zD, draft_tokens, tau, seed, round, logw_out, bonus_out, log
     _want(logw_out, torch.float64, (B, N), "logw_out")
     _want(bonus_out, torch.int32, (B, N), "bonus_out")
     _want(logw_prev, torch.float64, (B, N), "logw_prev")
+    _want(log_potential, torch.float64, (B, N), "log_potential")
     _want(tv_out, torch.float32, (B, N, R), "tv_out")
     _want(tokens_out, torch.int32, (B, N, R), "tokens_out")
     _want(lse_out, torch.float64, (B, N, R, 2), "lse_out")
     _want(lp_out, torch.float64, (B, N, K, 2), "lp_out")
     _check_err(dev_err)
     st = load().smcsd_score(_p(zT), _p(zD), _dtype(zT), B, N, K, V, ld, _p(draft_tokens),
-                            float(tau), int(seed), int(round), _p(logw_prev), _p(logw_out),
+                            float(tau), int(seed), int(round), _p(logw_prev),
+                            _p(log_potential), _p(logw_out),
                             _p(bonus_out), _p(tv_out), _p(tokens_out), _p(lse_out), _p(lp_out),
                             _p(dev_err), _stream(stream))
     _check("smcsd_score", st)
@@ -164,6 +169,24 @@ def smcsd_resample(logw, seed, round, ancestors_out, w_out=None, ess_out=None, d
     st = load().smcsd_resample(_p(logw), B, N, int(seed), int(round), _p(w_out), _p(ess_out),
                                _p(ancestors_out), _p(dev_err), _stream(stream))
     _check("smcsd_resample", st)
+
+
+def smcsd_resample_adaptive(logw, ess_frac, seed, round, ancestors_out, resampled_out=None,
+                            logw_next=None, w_out=None, ess_out=None, dev_err=None, stream=None):
+    """Resamples sequence b only where ESS < ess_frac * N; logw_next may be logw."""
+    B, N = logw.shape
+    _want(logw, torch.float64, (B, N), "logw")
+    _want(ancestors_out, torch.int32, (B, N), "ancestors_out")
+    _want(resampled_out, torch.int32, (B,), "resampled_out")
+    _want(logw_next, torch.float64, (B, N), "logw_next")
+    _want(w_out, torch.float64, (B, N), "w_out")
+    _want(ess_out, torch.float64, (B,), "ess_out")
+    _check_err(dev_err)
+    st = load().smcsd_resample_adaptive(_p(logw), B, N, float(ess_frac), int(seed), int(round),
+                                        _p(w_out), _p(ess_out), _p(ancestors_out),
+                                        _p(resampled_out), _p(logw_next), _p(dev_err),
+                                        _stream(stream))
+    _check("smcsd_resample_adaptive", st)
 
 
 def kv_pagetable_remap(pt_in, ancestors, pt_out, tok_in=None, tok_out=None, page_refcnt=None,

@@ -11,4 +11,4 @@ extern "C" const char* sd_status_string(sd_status s) {
   return "unknown status";
 }
 
-extern "C" int sd_version(void) { return 100; }
+extern "C" int sd_version(void) { return 200; }

@@ -4,9 +4,12 @@
 // "Faster LLM Inference via Sequential Monte Carlo", section 2 (resampling
 // step): particles with low importance weight are evicted and high-weight ones
 // duplicated to form the next round's N particles.  The scheme used here is
-// systematic resampling, run every round:
+// systematic resampling, every round or (adaptive, the usual SMC refinement
+// the page's section 5 extensions build on) only when ESS < ess_frac * N:
 //   W_j = exp(logw_j - max) / sum,  ESS = 1 / sum W_j^2,
 //   C_j = W_0 + ... + W_j,  U_i = (i + u0) / N,  a_i = min{ j : C_j > U_i }.
+// A sequence left alone keeps the identity ancestors and carries its
+// log-weights to the next round (logw_next = logw; 0 after a resample).
 // The order of every reduction is fixed, so results are bit-reproducible.
 #include <cuda_runtime.h>
 
@@ -83,9 +86,12 @@ __device__ double block_exclusive_scan_d(double v, double* scratch) {
 // scalar).  The running sum is a block-wide scan over chunks of T particles
 // with a carried offset.  Shared layout: [0, 40) reduction scratch, then the
 // N weights / running sums, both 16-byte aligned.
-__global__ void resample_kernel(const double* __restrict__ logw, int N, uint64_t seed,
+// logw_next may alias logw (each entry is read before the same thread writes
+// it), so neither carries __restrict__.
+__global__ void resample_kernel(const double* logw, int N, double ess_frac, uint64_t seed,
                                 uint64_t round, double* __restrict__ w_out,
                                 double* __restrict__ ess_out, int32_t* __restrict__ anc_out,
+                                int32_t* __restrict__ resampled_out, double* logw_next,
                                 uint32_t* dev_err) {
   extern __shared__ __align__(16) double sh_all[];
   double* scratch = sh_all;
@@ -107,9 +113,11 @@ __global__ void resample_kernel(const double* __restrict__ logw, int N, uint64_t
     for (int j = t; j < N; j += T) {
       if (w_out) w_out[(int64_t)b * N + j] = NAN;
       anc_out[(int64_t)b * N + j] = j;
+      if (logw_next) logw_next[(int64_t)b * N + j] = lw[j];
     }
     if (t == 0) {
       if (ess_out) ess_out[b] = NAN;
+      if (resampled_out) resampled_out[b] = 0;
       raise_err(dev_err, SD_DEV_NONFINITE);
     }
     return;
@@ -129,6 +137,16 @@ __global__ void resample_kernel(const double* __restrict__ logw, int N, uint64_t
     sq += W * W;
   }
   const double sumsq = block_sum_d(sq, scratch);
+  const double ess = 1.0 / sumsq;
+  if (t == 0 && ess_out) ess_out[b] = ess;
+  const bool resample = ess < ess_frac * (double)N;
+  if (t == 0 && resampled_out) resampled_out[b] = resample ? 1 : 0;
+  if (logw_next)
+    for (int j = t; j < N; j += T) logw_next[(int64_t)b * N + j] = resample ? 0.0 : lw[j];
+  if (!resample) {  // the weights carry: every particle is its own ancestor
+    for (int j = t; j < N; j += T) anc_out[(int64_t)b * N + j] = j;
+    return;
+  }
   // running sums C_j, chunk by chunk
   double carry = 0.0;
   for (int c0 = 0; c0 < N; c0 += T) {
@@ -140,7 +158,6 @@ __global__ void resample_kernel(const double* __restrict__ logw, int N, uint64_t
     carry += total;
   }
   __syncthreads();
-  if (t == 0 && ess_out) ess_out[b] = 1.0 / sumsq;
   const Stream st(seed, round, SD_STREAM_RESAMPLE);
   const double u0 = uniform_f64(st.at(0, (uint32_t)b).x);
   for (int i = t; i < N; i += T) {
@@ -159,20 +176,44 @@ __global__ void resample_kernel(const double* __restrict__ logw, int N, uint64_t
 
 using namespace smcsd;
 
-extern "C" sd_status smcsd_resample(const double* logw, int B, int N, uint64_t seed,
-                                    uint64_t round, double* w_out, double* ess_out,
-                                    int32_t* ancestors_out, uint32_t* dev_err, void* stream) {
-  if (B < 0 || N < 1) return SD_ERR_INVALID_ARG;
+namespace smcsd {
+static sd_status launch_resample(const double* logw, int B, int N, double ess_frac, uint64_t seed,
+                                 uint64_t round, double* w_out, double* ess_out,
+                                 int32_t* ancestors_out, int32_t* resampled_out,
+                                 double* logw_next, uint32_t* dev_err, void* stream) {
+  if (B < 0 || N < 1 || !(ess_frac >= 0.0)) return SD_ERR_INVALID_ARG;
   if (N > kResampleMaxN) return SD_ERR_UNSUPPORTED;
   if (B == 0) return SD_OK;
   if (!logw || !ancestors_out) return SD_ERR_INVALID_ARG;
   int threads = (N + 31) / 32 * 32;  // one particle per thread up to 1024
   if (threads > 1024) threads = 1024;
   const size_t smem = (size_t)(N + 40) * sizeof(double);
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute(resample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  resample_kernel<<<B, threads, smem, (cudaStream_t)stream>>>(logw, N, seed, round, w_out, ess_out,
-                                                             ancestors_out, dev_err);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(resample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess) {
+    cudaGetLastError();
+    return SD_ERR_CUDA;
+  }
+  resample_kernel<<<B, threads, smem, (cudaStream_t)stream>>>(
+      logw, N, ess_frac, seed, round, w_out, ess_out, ancestors_out, resampled_out, logw_next,
+      dev_err);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
   return SD_OK;
+}
+}  // namespace smcsd
+
+extern "C" sd_status smcsd_resample(const double* logw, int B, int N, uint64_t seed,
+                                    uint64_t round, double* w_out, double* ess_out,
+                                    int32_t* ancestors_out, uint32_t* dev_err, void* stream) {
+  return launch_resample(logw, B, N, INFINITY, seed, round, w_out, ess_out, ancestors_out, nullptr,
+                         nullptr, dev_err, stream);
+}
+
+extern "C" sd_status smcsd_resample_adaptive(const double* logw, int B, int N, double ess_frac,
+                                             uint64_t seed, uint64_t round, double* w_out,
+                                             double* ess_out, int32_t* ancestors_out,
+                                             int32_t* resampled_out, double* logw_next,
+                                             uint32_t* dev_err, void* stream) {
+  return launch_resample(logw, B, N, ess_frac, seed, round, w_out, ess_out, ancestors_out,
+                         resampled_out, logw_next, dev_err, stream);
 }

@@ -31,6 +31,7 @@ struct ScoreArgs {
   const int32_t* draft;  // [units, K]
   uint64_t seed, round;
   const double* logw_prev;
+  const double* log_potential;
   double* logw_out;
   float* tv_out;
   int32_t* bonus_out;

@@ -310,8 +310,11 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
   auto fetch_tokens = [&](int64_t u) -> int {
     return (lane_tokens && lane < a.K && u < a.units) ? a.draft[u * a.K + lane] : -1;
   };
+  // the weight carried in: the previous round's log-weight plus this round's
+  // log-potential of the particle (either may be absent)
   auto fetch_prev = [&](int64_t u) -> double {
-    return (a.logw_prev && u < a.units) ? a.logw_prev[u] : 0.0;
+    if (u >= a.units) return 0.0;
+    return (a.logw_prev ? a.logw_prev[u] : 0.0) + (a.log_potential ? a.log_potential[u] : 0.0);
   };
   int xs = -1, xs_next = fetch_tokens(unit);
   double lwp = 0.0, lwp_next = fetch_prev(unit);
@@ -877,7 +880,8 @@ using namespace smcsd;
 extern "C" sd_status smcsd_score(const void* zT, const void* zD, sd_dtype dt, int B, int N, int K,
                                  int V, int64_t ld, const int32_t* draft_tokens, float tau,
                                  uint64_t seed, uint64_t round, const double* logw_prev,
-                                 double* logw_out, int32_t* bonus_out, float* tv_out,
+                                 const double* log_potential, double* logw_out,
+                                 int32_t* bonus_out, float* tv_out,
                                  int32_t* tokens_out, double* lse_out, double* lp_out,
                                  uint32_t* dev_err, void* stream) {
   if (B < 0 || N < 1 || K < 0 || V < 1 || ld < V || !tau_ok(tau)) return SD_ERR_INVALID_ARG;
@@ -899,6 +903,7 @@ extern "C" sd_status smcsd_score(const void* zT, const void* zD, sd_dtype dt, in
   a.seed = seed;
   a.round = round;
   a.logw_prev = logw_prev;
+  a.log_potential = log_potential;
   a.logw_out = logw_out;
   a.tv_out = tv_out;
   a.bonus_out = bonus_out;

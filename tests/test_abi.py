@@ -37,28 +37,35 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     assert lib.status_string(lib.SD_OK) == "ok"
     assert "invalid" in lib.status_string(lib.SD_ERR_INVALID_ARG)
-    assert lib.version() >= 100
+    assert lib.version() >= 200
 
 
 def test_host_argument_checks_need_no_gpu():
     L = lib.load()
     vp = ctypes.c_void_p
     # N = 0 -> invalid before anything touches CUDA
-    assert L.smcsd_score(vp(1), vp(1), 1, 1, 0, 1, 10, 10, vp(1), 1.0, 0, 0, None, vp(1), vp(1),
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 0, 1, 10, 10, vp(1), 1.0, 0, 0, None, None, vp(1), vp(1),
                          None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
     # tau <= 0, ld < V
-    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 10, vp(1), 0.0, 0, 0, None, vp(1), vp(1),
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 10, vp(1), 0.0, 0, 0, None, None, vp(1), vp(1),
                          None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
-    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 9, vp(1), 1.0, 0, 0, None, vp(1), vp(1),
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 9, vp(1), 1.0, 0, 0, None, None, vp(1), vp(1),
                          None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
     # B = 0 is an empty batch: OK, nothing enqueued
-    assert L.smcsd_score(None, None, 1, 0, 1, 1, 10, 10, None, 1.0, 0, 0, None, None, None,
+    assert L.smcsd_score(None, None, 1, 0, 1, 1, 10, 10, None, 1.0, 0, 0, None, None, None, None,
                          None, None, None, None, None, None) == lib.SD_OK
     # missing required outputs
-    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 10, vp(1), 1.0, 0, 0, None, None, vp(1),
+    assert L.smcsd_score(vp(1), vp(1), 1, 1, 1, 1, 10, 10, vp(1), 1.0, 0, 0, None, None, None, vp(1),
                          None, None, None, None, None, None) == lib.SD_ERR_INVALID_ARG
     assert L.smcsd_resample(vp(1), 1, 0, 0, 0, None, None, vp(1), None, None) == lib.SD_ERR_INVALID_ARG
     assert L.smcsd_resample(vp(1), 1, 9000, 0, 0, None, None, vp(1), None, None) == lib.SD_ERR_UNSUPPORTED
+    for bad_frac in (float("nan"), -0.5):                           # ess_frac not >= 0
+        assert L.smcsd_resample_adaptive(vp(1), 1, 4, bad_frac, 0, 0, None, None, vp(1), None,
+                                         None, None, None) == lib.SD_ERR_INVALID_ARG
+    assert L.smcsd_resample_adaptive(vp(1), 1, 9000, 0.5, 0, 0, None, None, vp(1), None, None,
+                                     None, None) == lib.SD_ERR_UNSUPPORTED
+    assert L.smcsd_resample_adaptive(None, 0, 4, 0.5, 0, 0, None, None, None, None, None, None,
+                                     None) == lib.SD_OK                 # empty batch
     assert L.kv_pagetable_remap(vp(16), vp(16), 1, 1, 4, vp(16), vp(1), 2, None, None, 0, None,
                                 None) == lib.SD_ERR_INVALID_ARG     # tok_in without tok_out
     assert L.kv_pagetable_remap(vp(16), vp(16), 1, 1, 4, vp(16), None, 0, None, None, 0, None,

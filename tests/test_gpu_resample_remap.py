@@ -53,6 +53,68 @@ def test_resample_edge_cases():
     close(g["W"], o["W"], 1e-12, "W")
 
 
+def run_adaptive(logw, ess_frac, seed, rnd, in_place=False):
+    B, N = logw.shape
+    lw = to_dev(np.asarray(logw, dtype=np.float64))
+    anc = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    res = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    nxt = lw if in_place else torch.empty((B, N), dtype=torch.float64, device="cuda")
+    W = torch.empty((B, N), dtype=torch.float64, device="cuda")
+    ess = torch.empty((B,), dtype=torch.float64, device="cuda")
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    lib.smcsd_resample_adaptive(lw, ess_frac, seed, rnd, anc, resampled_out=res, logw_next=nxt,
+                                w_out=W, ess_out=ess, dev_err=err)
+    torch.cuda.synchronize()
+    return dict(anc=anc.cpu().numpy(), resampled=res.cpu().numpy(), logw_next=nxt.cpu().numpy(),
+                W=W.cpu().numpy(), ess=ess.cpu().numpy(), err=int(err.item()))
+
+
+@pytest.mark.parametrize("B,N,scale,frac", [(64, 4, 2.0, 0.5), (256, 32, 1.0, 0.5), (3, 1000, 0.3, 0.9),
+                                            (2, 8192, 5.0, 0.5), (40, 16, 1.0, 0.0),
+                                            (40, 16, 1.0, float("inf")), (9, 1, 1.0, 1.0)])
+@pytest.mark.parametrize("in_place", [False, True])
+def test_adaptive_resample_parity(B, N, scale, frac, in_place):
+    rng = np.random.default_rng(B * 7 + N)
+    # per-sequence spreads so some sequences fall below the threshold and some do not
+    logw = rng.standard_normal((B, N)) * scale * rng.uniform(0.1, 2.0, size=(B, 1))
+    g = run_adaptive(logw, frac, B + 1, N + 2, in_place)
+    o = oracle.smcsd_resample_adaptive(logw, frac, B + 1, N + 2)
+    close(g["W"], o["W"], 1e-12, "W")
+    close(g["ess"], o["ess"], 1e-9 * N, "ess")
+    # the trigger is a floating point comparison of ESS with frac * N: both sides
+    # take it in fp64; a sequence within rounding of the threshold may differ
+    near = np.abs(o["ess"] - frac * N) <= 1e-9 * N if np.isfinite(frac) else np.zeros(B, bool)
+    same = ~near
+    assert np.array_equal(g["resampled"][same], o["resampled"][same].astype(np.int32))
+    for b in np.flatnonzero(same):
+        if o["resampled"][b]:
+            discrete(g["anc"][b:b + 1], o["ancestors"][b:b + 1], o["margin"][b:b + 1], "ancestors")
+            assert np.all(g["logw_next"][b] == 0.0)
+        else:
+            assert np.array_equal(g["anc"][b], np.arange(N))
+            assert np.array_equal(g["logw_next"][b], logw[b])
+    assert g["err"] == 0
+    if frac == 0.0:
+        assert not g["resampled"].any()
+    if frac == float("inf"):
+        assert g["resampled"].all()
+        ref = run_resample(logw, B + 1, N + 2)
+        assert np.array_equal(g["anc"], ref["anc"])
+
+
+def test_adaptive_resample_faults():
+    logw = np.array([[0.0, np.nan, 1.0], [-np.inf, -np.inf, -np.inf], [0.0, 0.0, 9.0],
+                     [-np.inf, 3.0, -np.inf]])
+    g = run_adaptive(logw, 0.9, 1, 0)
+    o = oracle.smcsd_resample_adaptive(logw, 0.9, 1, 0)
+    assert g["err"] == o["err"] == oracle.DEV_NONFINITE
+    assert np.array_equal(g["resampled"], o["resampled"].astype(np.int32))
+    assert list(g["resampled"]) == [0, 0, 1, 1]
+    assert np.array_equal(g["anc"][:2], np.tile(np.arange(3), (2, 1)))
+    assert np.array_equal(g["logw_next"][:2], logw[:2], equal_nan=True)
+    assert np.all(g["anc"][3] == 1)
+
+
 def run_remap(pt, anc, num_pages=None, tok=None):
     B, N, P = pt.shape
     pti = to_dev(pt.astype(np.int32))

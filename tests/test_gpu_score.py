@@ -13,7 +13,8 @@ from tests.parity import TOL_LOGW, TOL_LSE, TOL_TV, bf16_dev, close, discrete, r
 pytestmark = [pytest.mark.gpu, requires_gpu]
 
 
-def run_score(zT, zD, x, tau, seed, rnd, dtype="bf16", logw_prev=None, ld=None):
+def run_score(zT, zD, x, tau, seed, rnd, dtype="bf16", logw_prev=None, ld=None,
+              log_potential=None):
     B, N, R, V = zT.shape
     K = R - 1
     dev = "cuda"
@@ -37,8 +38,9 @@ def run_score(zT, zD, x, tau, seed, rnd, dtype="bf16", logw_prev=None, ld=None):
         lp=torch.empty((B, N, K, 2), dtype=torch.float64, device=dev),
         err=torch.zeros((1,), dtype=torch.int32, device=dev))
     prev = None if logw_prev is None else to_dev(np.asarray(logw_prev, dtype=np.float64))
+    phi = None if log_potential is None else to_dev(np.asarray(log_potential, dtype=np.float64))
     lib.smcsd_score(t, d, xs, tau, seed, rnd, out["logw"], out["bonus"], logw_prev=prev,
-                    tv_out=out["tv"], tokens_out=out["tokens"], lse_out=out["lse"],
+                    log_potential=phi, tv_out=out["tv"], tokens_out=out["tokens"], lse_out=out["lse"],
                     lp_out=out["lp"], dev_err=out["err"])
     torch.cuda.synchronize()
     res = {k: v.cpu().numpy() for k, v in out.items()}
@@ -236,3 +238,28 @@ def test_full_size_config_sampled(name, seqs):
         discrete(out_bonus[b:b + 1].cpu().numpy(), o["bonus"], o["bonus_margin"], f"{name}[{b}].bonus")
     del d
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("with_prev", [False, True])
+def test_log_potential(with_prev):
+    """A per-particle log-potential (reward-weighted / constrained target) adds
+    to the carried weight; -inf rules a particle out without an error."""
+    rng = np.random.default_rng(41)
+    B, N, K, V = 3, 8, 4, 3000
+    zT, zD, x = rand_case(rng, B, N, K, V)
+    phi = rng.standard_normal((B, N)) * 2.0
+    phi[1, 3] = -np.inf
+    prev = rng.standard_normal((B, N)) if with_prev else None
+    g = run_score(zT, zD, x, 0.8, 12, 3, logw_prev=prev, log_potential=phi)
+    o = oracle.smcsd_score(zT, zD, x, 0.8, 12, 3, logw_prev=prev, log_potential=phi)
+    assert g["logw"][1, 3] == -np.inf
+    close(np.where(np.isinf(g["logw"]), 0, g["logw"]), np.where(np.isinf(o["logw"]), 0, o["logw"]),
+          TOL_LOGW, "logw")
+    compare({**g, "logw": np.nan_to_num(g["logw"], neginf=0)},
+            {**o, "logw": np.nan_to_num(o["logw"], neginf=0)}, "potential")
+    # the potential shifts nothing but the weight
+    g0 = run_score(zT, zD, x, 0.8, 12, 3, logw_prev=prev)
+    for k in ("tv", "lse", "lp", "bonus", "tokens"):
+        assert np.array_equal(g[k], g0[k]), k
+    fin = np.isfinite(phi)
+    assert np.allclose((g["logw"] - g0["logw"])[fin], phi[fin], atol=1e-12, rtol=0)

@@ -12,8 +12,9 @@ Sources (summaries on gist.science; each function cites its passage):
     importance weights, evict/duplicate resampling, bonus token, KV page
     metadata copy (section 2, Methodology).
   * METASD (multi-drafter speculative decoding) -- Block Divergence reward built
-    on the total-variation distance between drafter and target distributions
-    (section 2, Methodology); standard SD verification (section 1).
+    on the total-variation distance between drafter and target distributions,
+    drafter selection by an upper-confidence-bound bandit (section 2,
+    Methodology); standard SD verification (section 1).
   * STAND (stochastic adaptive n-gram drafting) -- Gumbel-Top-K sampling without
     replacement from stored top-10 (index, probability) rows (Methodology,
     items 1 and 2); stochastic drafting from a distribution rather than its
@@ -35,3 +36,4 @@ from .pagetable import kv_pagetable_remap  # noqa: F401
 from .verify import sd_verify_reject, accept_probability, residual_distribution  # noqa: F401
 from .topk import gumbel_topk, gumbel_topk_sparse  # noqa: F401
 from .draft import sd_draft_sample  # noqa: F401
+from .bandit import metasd_ucb_step, block_reward, ucb_choice, DEV_ARM_OOB, REWARD_BD, REWARD_BE  # noqa: F401,E501

@@ -9,7 +9,8 @@
  *             evict/duplicate resampling, bonus token, KV page metadata copy)
  *             and section 1 (standard SD and its rejection step).
  *   [METASD]  METASD (multi-drafter speculative decoding), section 2
- *             (Block Divergence reward built on total-variation distance).
+ *             (Block Divergence reward built on total-variation distance,
+ *             drafter selection by a UCB bandit).
  *   [STAND]   STAND (stochastic adaptive n-gram drafting), Methodology items
  *             1 (top-10 logit n-gram store) and 2 (Gumbel-Top-K sampling).
  *
@@ -69,9 +70,14 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_DEV_PAGE_OOB 8u       /* page id outside [0, num_pages) and != -1   */
 #define SD_DEV_ANCESTOR_OOB 16u  /* ancestor index outside [0, N)              */
 #define SD_DEV_TIMEOUT 32u       /* an internal bounded wait gave up           */
+#define SD_DEV_ARM_OOB 64u       /* bandit: an arm index outside [-1, M)       */
 /* With SD_DEV_TIMEOUT, smcsd_score also sets one of bits 8..15 naming the
  * wait that gave up (diagnostic only; outputs of that call are invalid). */
 #define SD_DEV_WAIT_SITE_MASK 0xFF00u
+
+/* Reward of the drafter-selection bandit (sd_metasd_ucb). */
+#define SD_REWARD_BD 0 /* Block Divergence: 1 - mean TV over the K drafted positions */
+#define SD_REWARD_BE 1 /* Block Efficiency: accepted tokens / K                     */
 
 /* Philox stream tags. */
 #define SD_STREAM_BONUS 1u
@@ -270,6 +276,40 @@ SMCSD_API sd_status sd_draft_sample(const void* zD, sd_dtype dt, int rows, int V
                                     float tau, uint64_t seed, uint64_t round, uint32_t row0,
                                     int32_t* tokens_out, float* logq_out, uint32_t* dev_err,
                                     void* stream);
+
+/*
+ * sd_metasd_ucb -- one round of drafter selection for B sequences, each with
+ * its own M-armed bandit ([METASD] section 2: a multi-armed bandit picks the
+ * drafter of each round; its reward is the Block Divergence, built on the TV
+ * distance between drafter and target, or the Block Efficiency, the
+ * accepted-token count; MetaSD-UCB is an upper-confidence-bound rule).  The
+ * page gives no formula; the rule here is UCB1 with rewards in [0, 1]:
+ *   reward  BD = 1 - (1/K) sum_{k<K} tv[b, k]   (fp64, summed in k order)
+ *           BE = accepted_len[b] / K
+ *   update  pulls[b, a] += 1, sums[b, a] += reward, a = arm_in[b]
+ *           (nothing when arm_in[b] == -1: no arm used yet)
+ *   choose  arm_out[b] = the lowest arm never pulled, else
+ *           argmax_i sums/pulls + sqrt(c * ln(t) / pulls), t = sum_i pulls,
+ *           ties to the lowest i.  c = 2 is the textbook UCB1 bonus.
+ * tv            device fp32 [B, ld_tv], ld_tv >= K (the per-position TV of
+ *               sd_verify_reject); needed for BD, ignored for BE.
+ * accepted_len  device int32 [B]; needed for BE, ignored for BD.
+ * arm_in        device int32 [B]: the arm each sequence used this round, or -1.
+ * pulls, sums   device int32 / fp64 [B, M]: the bandit state, caller-owned,
+ *               zero to start, updated in place.
+ * arm_out       device int32 [B] (may alias arm_in: each thread reads its own
+ *               entry first).
+ * reward_out    device fp64 [B] or NULL: the reward credited (NaN if none).
+ * Requirements: B >= 0, K >= 1, 1 <= M <= 4096, 0 <= c < inf,
+ *   reward_kind SD_REWARD_BD or SD_REWARD_BE.
+ * Faults: arm_in outside [-1, M) -> SD_DEV_ARM_OOB, no update; a NaN TV or an
+ *   accepted length outside [0, K] -> SD_DEV_NONFINITE, no update.  The
+ *   next arm is chosen in both cases.
+ */
+SMCSD_API sd_status sd_metasd_ucb(const float* tv, int64_t ld_tv, const int32_t* accepted_len,
+                                  const int32_t* arm_in, int B, int K, int M, int reward_kind,
+                                  double c, int32_t* pulls, double* sums, int32_t* arm_out,
+                                  double* reward_out, uint32_t* dev_err, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 SMCSD_API const char* sd_status_string(sd_status s);

@@ -22,8 +22,9 @@ Readings (the plainest ones the prose supports):
 One call of ``metasd_ucb_step`` is one round for B sequences: the reward of the
 arm each sequence used (arm_in = -1: no arm yet) updates its (pulls, sums) and
 the rule picks the arm of the next round.  A reward that is not finite (a NaN
-TV row) leaves the state untouched and raises the non-finite error bit; an
-arm_in outside [-1, M) raises the arm error bit and is ignored.
+TV row, an accepted length outside [0, K]) leaves the state untouched and
+raises the non-finite error bit; an arm_in outside [-1, M) raises the arm
+error bit and is ignored.
 
 Parity status: pinned by the textbook UCB1 values on a worked example, the
 pull-every-arm-first rule, the BD / BE closed forms on hand-made rows, and by
@@ -46,6 +47,8 @@ def block_reward(tv_row, accepted_len, K, kind):
     if kind == REWARD_BD:
         tv = [float(t) for t in tv_row[:K]]
         return 1.0 - sum(tv) / K
+    if not 0 <= int(accepted_len) <= K:
+        return math.nan      # not a block length: treated as a faulty round
     return float(accepted_len) / K
 
 

@@ -19,11 +19,12 @@ LIB_PATH = os.path.join(_HERE, "libsmcsd.so")
 SD_OK, SD_ERR_INVALID_ARG, SD_ERR_CUDA, SD_ERR_UNSUPPORTED = 0, 1, 2, 3
 SD_F32, SD_BF16 = 0, 1
 DEV_TOKEN_OOB, DEV_NONFINITE, DEV_ZERO_RESIDUAL = 1, 2, 4
-DEV_PAGE_OOB, DEV_ANCESTOR_OOB, DEV_TIMEOUT = 8, 16, 32
+DEV_PAGE_OOB, DEV_ANCESTOR_OOB, DEV_TIMEOUT, DEV_ARM_OOB = 8, 16, 32, 64
+REWARD_BD, REWARD_BE = 0, 1
 
 EXPORTS = ("smcsd_score", "smcsd_resample", "smcsd_resample_adaptive", "kv_pagetable_remap",
            "sd_verify_reject", "gumbel_topk", "gumbel_topk_sparse", "sd_draft_sample",
-           "sd_status_string", "sd_version")
+           "sd_metasd_ucb", "sd_status_string", "sd_version")
 
 _lib = None
 
@@ -57,7 +58,8 @@ def load():
     L.gumbel_topk_sparse.argtypes = [vp, vp, i32, i32, i32, f32, u64, u64, vp, vp, vp]
     L.sd_draft_sample.argtypes = [vp, i32, i32, i32, i64, f32, u64, u64, ctypes.c_uint32, vp, vp,
                                   vp, vp]
-    for name in EXPORTS[:8]:
+    L.sd_metasd_ucb.argtypes = [vp, i64, vp, vp, i32, i32, i32, i32, f64, vp, vp, vp, vp, vp, vp]
+    for name in EXPORTS[:9]:
         getattr(L, name).restype = ctypes.c_int
     L.sd_status_string.argtypes = [ctypes.c_int]
     L.sd_status_string.restype = ctypes.c_char_p
@@ -266,3 +268,30 @@ def sd_draft_sample(zD, tau, seed, round, tokens_out, logq_out=None, row0=0, dev
                                 int(row0), _p(tokens_out), _p(logq_out), _p(dev_err),
                                 _stream(stream))
     _check("sd_draft_sample", st)
+
+
+def sd_metasd_ucb(arm_in, pulls, sums, arm_out, K, tv=None, accepted_len=None,
+                  reward_kind=REWARD_BD, c=2.0, reward_out=None, dev_err=None, stream=None):
+    """One drafter-selection round for B sequences; pulls int32 / sums fp64 [B, M]
+    are updated in place.  tv: fp32 [B, >=K] (BD); accepted_len: int32 [B] (BE)."""
+    B, M = pulls.shape
+    _want(arm_in, torch.int32, (B,), "arm_in")
+    _want(arm_out, torch.int32, (B,), "arm_out")
+    _want(pulls, torch.int32, (B, M), "pulls")
+    _want(sums, torch.float64, (B, M), "sums")
+    _want(reward_out, torch.float64, (B,), "reward_out")
+    ld = 0
+    if tv is not None:
+        if tv.dim() != 2 or tv.shape[0] != B or tv.dtype != torch.float32 or not tv.is_cuda \
+                or tv.stride(1) != 1:
+            raise ValueError(f"tv: expected CUDA float32 [{B}, >={K}] with unit inner stride")
+        ld = tv.stride(0) if B > 1 else tv.shape[1]
+        if tv.shape[1] < K:
+            raise ValueError("tv has fewer than K columns")
+    if accepted_len is not None:
+        _want(accepted_len, torch.int32, (B,), "accepted_len")
+    _check_err(dev_err)
+    st = load().sd_metasd_ucb(_p(tv), ld, _p(accepted_len), _p(arm_in), B, int(K), M,
+                              int(reward_kind), float(c), _p(pulls), _p(sums), _p(arm_out),
+                              _p(reward_out), _p(dev_err), _stream(stream))
+    _check("sd_metasd_ucb", st)

@@ -80,6 +80,16 @@ def test_host_argument_checks_need_no_gpu():
                                 None) == lib.SD_ERR_INVALID_ARG     # k > L
     assert L.sd_draft_sample(vp(1), 1, 4, 10, 10, 0.0, 0, 0, 0, vp(1), None, None,
                              None) == lib.SD_ERR_INVALID_ARG        # tau <= 0
+    assert L.sd_metasd_ucb(vp(1), 2, None, vp(1), 1, 4, 2, 0, 2.0, vp(1), vp(1), vp(1), None,
+                           None, None) == lib.SD_ERR_INVALID_ARG    # ld_tv < K
+    assert L.sd_metasd_ucb(None, 0, None, vp(1), 1, 4, 2, 1, 2.0, vp(1), vp(1), vp(1), None,
+                           None, None) == lib.SD_ERR_INVALID_ARG    # BE without accepted_len
+    assert L.sd_metasd_ucb(vp(1), 4, None, vp(1), 1, 4, 2, 0, -1.0, vp(1), vp(1), vp(1), None,
+                           None, None) == lib.SD_ERR_INVALID_ARG    # c < 0
+    assert L.sd_metasd_ucb(vp(1), 4, None, vp(1), 1, 4, 2, 2, 2.0, vp(1), vp(1), vp(1), None,
+                           None, None) == lib.SD_ERR_INVALID_ARG    # unknown reward kind
+    assert L.sd_metasd_ucb(None, 0, None, None, 0, 4, 2, 0, 2.0, None, None, None, None, None,
+                           None) == lib.SD_OK                        # empty batch
     assert L.sd_draft_sample(vp(1), 1, 4, 10, 10, 1.0, 0, 0, 0xFFFFFFFE, vp(1), None, None,
                              None) == lib.SD_ERR_INVALID_ARG        # row ids past 2^32
     assert L.sd_draft_sample(None, 1, 0, 10, 10, 1.0, 0, 0, 0, None, None, None,

@@ -39,6 +39,7 @@ def test_rewards_closed_form():
     assert oracle.block_reward(tv, 3, 4, REWARD_BE) == 0.75
     assert oracle.block_reward(np.zeros(4), 0, 4, REWARD_BD) == 1.0
     assert oracle.block_reward(np.ones(4), 4, 4, REWARD_BD) == 0.0
+    assert math.isnan(oracle.block_reward(tv, 5, 4, REWARD_BE))
 
 
 def test_step_updates_the_used_arm_only():

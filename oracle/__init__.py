@@ -15,8 +15,9 @@ Sources (summaries on gist.science; each function cites its passage):
     on the total-variation distance between drafter and target distributions,
     drafter selection by an upper-confidence-bound bandit (section 2,
     Methodology); standard SD verification (section 1).
-  * STAND (stochastic adaptive n-gram drafting) -- Gumbel-Top-K sampling without
-    replacement from stored top-10 (index, probability) rows (Methodology,
+  * STAND (stochastic adaptive n-gram drafting) -- the logit n-gram store
+    (top-10 (index, probability) rows, weighted-average merge, truncation) and
+    Gumbel-Top-K sampling without replacement from its rows (Methodology,
     items 1 and 2); stochastic drafting from a distribution rather than its
     argmax (Methodology, item 1).
 
@@ -37,3 +38,4 @@ from .verify import sd_verify_reject, accept_probability, residual_distribution 
 from .topk import gumbel_topk, gumbel_topk_sparse  # noqa: F401
 from .draft import sd_draft_sample  # noqa: F401
 from .bandit import metasd_ucb_step, block_reward, ucb_choice, DEV_ARM_OOB, REWARD_BD, REWARD_BE  # noqa: F401,E501
+from .ngram import NgramStore, observe_topk, merge as ngram_merge  # noqa: F401

@@ -45,8 +45,9 @@ KEY_MAX_ID = 1 << 20
 
 def observe_topk(z, tau, k, rows=None):
     """The k most likely entries of softmax(z[r] / tau) per row r (or per r in
-    rows): idx [U, k] int (ties to the lower index; -1 past V), prob [U, k]
-    fp32 (0 past V).  Non-finite rows (NaN / +inf / all -inf) give idx -1,
+    rows): idx [U, k] int (ties to the lower index; -1 past V and in place of
+    -inf entries, which have probability 0 and are not stored), prob [U, k]
+    fp32 (0 where idx is -1).  Non-finite rows (NaN / +inf / all -inf) give idx -1,
     prob NaN and the non-finite error bit."""
     z = np.asarray(z)
     rows = np.arange(z.shape[0]) if rows is None else np.asarray(rows)
@@ -62,6 +63,7 @@ def observe_topk(z, tau, k, rows=None):
             continue
         a, lse = row_log_softmax(zr, tau)
         order = np.lexsort((np.arange(zr.shape[0]), -zr))[:k]  # z order = p order
+        order = order[np.isfinite(zr[order])]   # -inf entries have probability 0: not stored
         idx[u, :order.shape[0]] = order
         prob[u, :order.shape[0]] = np.exp(a[order] - lse).astype(np.float32)
     return idx, prob, err

@@ -84,7 +84,7 @@ def test_observe_topk_matches_a_sort_of_the_softmax():
         assert idx[r].tolist() == order
         assert np.allclose(prob[r], p[order], rtol=1e-6, atol=0)
     assert idx[1, :3].tolist() == [10, 20, 30]
-    assert idx[2, 0] == 7 and prob[2, 0] == 1.0
+    assert idx[2].tolist() == [7] + [-1] * 9 and prob[2, 0] == 1.0 and np.all(prob[2, 1:] == 0)
     assert idx[3].tolist() == [-1] * 10 and np.isnan(prob[3]).all()
     # rows past the first: row selection
     idx2, prob2, _ = observe_topk(z, 0.7, 10, rows=[4, 0])

@@ -42,6 +42,7 @@
 #ifndef SMCSD_H_
 #define SMCSD_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -71,6 +72,7 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_DEV_ANCESTOR_OOB 16u  /* ancestor index outside [0, N)              */
 #define SD_DEV_TIMEOUT 32u       /* an internal bounded wait gave up           */
 #define SD_DEV_ARM_OOB 64u       /* bandit: an arm index outside [-1, M)       */
+#define SD_DEV_TABLE_FULL 128u   /* n-gram store: no free slot for a new key   */
 /* With SD_DEV_TIMEOUT, smcsd_score also sets one of bits 8..15 naming the
  * wait that gave up (diagnostic only; outputs of that call are invalid). */
 #define SD_DEV_WAIT_SITE_MASK 0xFF00u
@@ -310,6 +312,89 @@ SMCSD_API sd_status sd_metasd_ucb(const float* tv, int64_t ld_tv, const int32_t*
                                   const int32_t* arm_in, int B, int K, int M, int reward_kind,
                                   double c, int32_t* pulls, double* sums, int32_t* arm_out,
                                   double* reward_out, uint32_t* dev_err, void* stream);
+
+/*
+ * Logit n-gram store ([STAND] Methodology item 1): per observed n-gram, the
+ * next-token distribution reduced to its k most likely (index, probability)
+ * pairs; a repeated n-gram merges the stored and the new row by a weighted
+ * average (an unstored index counts as probability 0) and cuts the result
+ * back to the k largest, so each n-gram costs fixed memory.  Rows feed
+ * gumbel_topk_sparse (stochastic drafting, item 2).  Readings of the page:
+ *   - an observation is softmax(z / tau) at one position; its k largest
+ *     entries (ties to the lower index; -inf entries are not stored) keep
+ *     their probabilities under the full softmax, rounded to fp32;
+ *   - the average weighs by occurrence count c:
+ *       p_new(v) = (c * p_old(v) + p_obs(v)) / (c + 1)
+ *     in fp64 with each operation rounded once, then rounded to fp32; the k
+ *     largest results (ties to the lower index) are stored in that order,
+ *     unused entries as (-1, 0); the count becomes c + 1;
+ *   - observations of one n-gram within a call apply in their batch order.
+ * The table is one caller-owned device buffer of ngram_table_bytes(C, k)
+ * bytes, 16-byte aligned, zeroed by ngram_table_clear before first use:
+ *   keys u64 [C] | counts i32 [C] | idx i32 [C][k] | prob f32 [C][k];
+ * capacity C a power of two in [32, 2^40]; 1 <= k <= 16.  A key is the exact
+ * n-gram (1 <= n <= 3 token ids in [0, 2^20)); slots are found by linear
+ * probing from a hash of the key.  Nothing is ever deleted.
+ */
+/* Bytes of a table of C slots with k entries each (0 if C or k is invalid). */
+SMCSD_API size_t ngram_table_bytes(int64_t capacity, int k);
+/* Bytes of the workspace ngram_store_update needs for U observations (0 if
+ * U is outside [0, 16384]). */
+SMCSD_API size_t ngram_workspace_bytes(int U);
+/* Zeroes the table (every slot empty).  Enqueued on stream. */
+SMCSD_API sd_status ngram_table_clear(void* table, int64_t capacity, int k, void* stream);
+
+/*
+ * ngram_observe_topk -- the observation rows: for u < U, with r = row_ids[u]
+ * (or u when row_ids is NULL),
+ *   idx_out[u, :]  = the k largest entries of z[r, :] (ties to the lower
+ *                    index; finite entries only; -1 past them),
+ *   prob_out[u, :] = exp(z[r, v] / tau - logsumexp_w(z[r, w] / tau)) (0 past
+ *                    them), fp32.
+ * z         device [rows, V] at row stride ld, dtype dt.
+ * row_ids   device int32 [U] or NULL (then U <= rows).
+ * idx_out   device int32 [U, k];  prob_out device fp32 [U, k].
+ * Requirements: rows, U >= 0; V >= 1; ld >= V; 1 <= k <= 16; tau > 0 finite.
+ * Faults: a row with NaN / +inf or all -inf -> SD_DEV_NONFINITE, ids -1,
+ *   prob NaN; a row id outside [0, rows) -> SD_DEV_TOKEN_OOB, same outputs.
+ */
+SMCSD_API sd_status ngram_observe_topk(const void* z, sd_dtype dt, int rows, int V, int64_t ld,
+                                       const int32_t* row_ids, int U, int k, float tau,
+                                       int32_t* idx_out, float* prob_out, uint32_t* dev_err,
+                                       void* stream);
+
+/*
+ * ngram_store_update -- merges U observations into the table, in batch order
+ * for equal n-grams.
+ * ctx        device int32 [U, n]: the n-gram preceding each observation.
+ * idx, prob  device int32 / fp32 [U, k]: observation rows (ngram_observe_topk
+ *            output; -1 entries are empty).
+ * workspace  device, >= ngram_workspace_bytes(U) bytes, 4-byte aligned,
+ *            caller-owned scratch (no initial contents needed); calls that
+ *            share a workspace or a table must not overlap on the GPU.
+ * Requirements: 1 <= n <= 3; 0 <= U <= 16384 (more -> SD_ERR_UNSUPPORTED).
+ * Faults: a context id outside [0, 2^20) -> SD_DEV_TOKEN_OOB, that
+ *   observation skipped; a row with a NaN / infinite / negative probability
+ *   or a repeated index -> SD_DEV_NONFINITE, skipped; no free slot for a new
+ *   n-gram -> SD_DEV_TABLE_FULL, its observations skipped.
+ */
+SMCSD_API sd_status ngram_store_update(void* table, int64_t capacity, int k, const int32_t* ctx,
+                                       int n, const int32_t* idx, const float* prob, int U,
+                                       void* workspace, size_t workspace_bytes, uint32_t* dev_err,
+                                       void* stream);
+
+/*
+ * ngram_store_lookup -- the stored rows of Q n-grams.
+ * ctx        device int32 [Q, n].
+ * idx_out    device int32 [Q, k] (-1 where absent); prob_out device fp32
+ *            [Q, k] (0 where absent): ready for gumbel_topk_sparse (L = k).
+ * count_out  device int32 [Q] or NULL: observations merged (0 if absent).
+ * Faults: a context id outside [0, 2^20) -> SD_DEV_TOKEN_OOB, reported absent.
+ */
+SMCSD_API sd_status ngram_store_lookup(const void* table, int64_t capacity, int k,
+                                       const int32_t* ctx, int n, int Q, int32_t* idx_out,
+                                       float* prob_out, int32_t* count_out, uint32_t* dev_err,
+                                       void* stream);
 
 /* Human-readable name of a status code (static storage). */
 SMCSD_API const char* sd_status_string(sd_status s);

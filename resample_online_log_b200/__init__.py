@@ -19,12 +19,14 @@ LIB_PATH = os.path.join(_HERE, "libsmcsd.so")
 SD_OK, SD_ERR_INVALID_ARG, SD_ERR_CUDA, SD_ERR_UNSUPPORTED = 0, 1, 2, 3
 SD_F32, SD_BF16 = 0, 1
 DEV_TOKEN_OOB, DEV_NONFINITE, DEV_ZERO_RESIDUAL = 1, 2, 4
-DEV_PAGE_OOB, DEV_ANCESTOR_OOB, DEV_TIMEOUT, DEV_ARM_OOB = 8, 16, 32, 64
+DEV_PAGE_OOB, DEV_ANCESTOR_OOB, DEV_TIMEOUT, DEV_ARM_OOB, DEV_TABLE_FULL = 8, 16, 32, 64, 128
 REWARD_BD, REWARD_BE = 0, 1
 
 EXPORTS = ("smcsd_score", "smcsd_resample", "smcsd_resample_adaptive", "kv_pagetable_remap",
            "sd_verify_reject", "gumbel_topk", "gumbel_topk_sparse", "sd_draft_sample",
-           "sd_metasd_ucb", "sd_status_string", "sd_version")
+           "sd_metasd_ucb", "ngram_table_clear", "ngram_observe_topk", "ngram_store_update",
+           "ngram_store_lookup", "ngram_table_bytes", "ngram_workspace_bytes", "sd_status_string",
+           "sd_version")
 
 _lib = None
 
@@ -59,7 +61,16 @@ def load():
     L.sd_draft_sample.argtypes = [vp, i32, i32, i32, i64, f32, u64, u64, ctypes.c_uint32, vp, vp,
                                   vp, vp]
     L.sd_metasd_ucb.argtypes = [vp, i64, vp, vp, i32, i32, i32, i32, f64, vp, vp, vp, vp, vp, vp]
-    for name in EXPORTS[:9]:
+    L.ngram_table_clear.argtypes = [vp, i64, i32, vp]
+    L.ngram_observe_topk.argtypes = [vp, i32, i32, i32, i64, vp, i32, i32, f32, vp, vp, vp, vp]
+    L.ngram_store_update.argtypes = [vp, i64, i32, vp, i32, vp, vp, i32, vp, ctypes.c_size_t, vp,
+                                     vp]
+    L.ngram_store_lookup.argtypes = [vp, i64, i32, vp, i32, i32, vp, vp, vp, vp, vp]
+    L.ngram_table_bytes.argtypes = [i64, i32]
+    L.ngram_table_bytes.restype = ctypes.c_size_t
+    L.ngram_workspace_bytes.argtypes = [i32]
+    L.ngram_workspace_bytes.restype = ctypes.c_size_t
+    for name in EXPORTS[:13]:
         getattr(L, name).restype = ctypes.c_int
     L.sd_status_string.argtypes = [ctypes.c_int]
     L.sd_status_string.restype = ctypes.c_char_p
@@ -295,3 +306,92 @@ def sd_metasd_ucb(arm_in, pulls, sums, arm_out, K, tv=None, accepted_len=None,
                               int(reward_kind), float(c), _p(pulls), _p(sums), _p(arm_out),
                               _p(reward_out), _p(dev_err), _stream(stream))
     _check("sd_metasd_ucb", st)
+
+
+def ngram_table_bytes(capacity, k):
+    return load().ngram_table_bytes(int(capacity), int(k))
+
+
+def ngram_workspace_bytes(U):
+    return load().ngram_workspace_bytes(int(U))
+
+
+def _table(table, capacity, k):
+    need = ngram_table_bytes(capacity, k)
+    if need == 0:
+        raise ValueError(f"invalid n-gram table shape: capacity={capacity}, k={k}")
+    if table.dtype != torch.uint8 or table.dim() != 1 or table.numel() < need or not table.is_cuda \
+            or not table.is_contiguous():
+        raise ValueError(f"table: expected a contiguous CUDA uint8 buffer of >= {need} bytes")
+
+
+def ngram_table_clear(table, capacity, k, stream=None):
+    _table(table, capacity, k)
+    _check("ngram_table_clear", load().ngram_table_clear(_p(table), int(capacity), int(k),
+                                                         _stream(stream)))
+
+
+def ngram_observe_topk(z, k, tau, idx_out, prob_out, row_ids=None, dev_err=None, stream=None):
+    """z: [rows, V] (bf16 or fp32); row_ids int32 [U] or None (U = rows)."""
+    rows = z.shape[0]
+    V, ld = _rows_view(z, (rows,))
+    U = rows if row_ids is None else row_ids.shape[0]
+    _want(row_ids, torch.int32, (U,), "row_ids")
+    _want(idx_out, torch.int32, (U, k), "idx_out")
+    _want(prob_out, torch.float32, (U, k), "prob_out")
+    _check_err(dev_err)
+    st = load().ngram_observe_topk(_p(z), _dtype(z), rows, V, ld, _p(row_ids), U, int(k),
+                                   float(tau), _p(idx_out), _p(prob_out), _p(dev_err),
+                                   _stream(stream))
+    _check("ngram_observe_topk", st)
+
+
+def ngram_store_update(table, capacity, k, ctx, idx, prob, workspace, dev_err=None, stream=None):
+    """ctx int32 [U, n]; idx int32 / prob fp32 [U, k]; workspace: CUDA uint8 of
+    >= ngram_workspace_bytes(U) bytes."""
+    _table(table, capacity, k)
+    U, n = ctx.shape
+    _want(ctx, torch.int32, (U, n), "ctx")
+    _want(idx, torch.int32, (U, k), "idx")
+    _want(prob, torch.float32, (U, k), "prob")
+    if workspace.dtype != torch.uint8 or not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace: expected a contiguous CUDA uint8 buffer")
+    _check_err(dev_err)
+    st = load().ngram_store_update(_p(table), int(capacity), int(k), _p(ctx), n, _p(idx), _p(prob),
+                                   U, _p(workspace), workspace.numel(), _p(dev_err),
+                                   _stream(stream))
+    _check("ngram_store_update", st)
+
+
+def ngram_store_lookup(table, capacity, k, ctx, idx_out, prob_out, count_out=None, dev_err=None,
+                       stream=None):
+    _table(table, capacity, k)
+    Q, n = ctx.shape
+    _want(ctx, torch.int32, (Q, n), "ctx")
+    _want(idx_out, torch.int32, (Q, k), "idx_out")
+    _want(prob_out, torch.float32, (Q, k), "prob_out")
+    _want(count_out, torch.int32, (Q,), "count_out")
+    _check_err(dev_err)
+    st = load().ngram_store_lookup(_p(table), int(capacity), int(k), _p(ctx), n, Q, _p(idx_out),
+                                   _p(prob_out), _p(count_out), _p(dev_err), _stream(stream))
+    _check("ngram_store_lookup", st)
+
+
+class NgramTable:
+    """A logit n-gram store on the current CUDA device: the table buffer and an
+    update workspace held as torch tensors, cleared on creation."""
+
+    def __init__(self, capacity, k=10, max_update=16384, device="cuda"):
+        self.capacity, self.k = int(capacity), int(k)
+        self.table = torch.empty((ngram_table_bytes(capacity, k),), dtype=torch.uint8, device=device)
+        self.workspace = torch.empty((ngram_workspace_bytes(max_update),), dtype=torch.uint8,
+                                     device=device)
+        ngram_table_clear(self.table, capacity, k)
+
+    def update(self, ctx, idx, prob, dev_err=None, stream=None):
+        ngram_store_update(self.table, self.capacity, self.k, ctx, idx, prob, self.workspace,
+                           dev_err=dev_err, stream=stream)
+
+    def lookup(self, ctx, idx_out, prob_out, count_out=None, dev_err=None, stream=None):
+        ngram_store_lookup(self.table, self.capacity, self.k, ctx, idx_out, prob_out,
+                           count_out=count_out, dev_err=dev_err, stream=stream)

@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "rowload.cuh"
 
 namespace smcsd {
 
@@ -26,13 +27,7 @@ constexpr int kTopkMax = 16;     // k <= 16
 constexpr int kListMax = 17;     // longest per-thread list (k + 1)
 constexpr int kTopkThreads = 512;
 constexpr int kCandCap = 1024;   // candidates gathered per row
-
-// Order-preserving map of floats to signed ints (for atomicMax on a threshold).
-__device__ __forceinline__ int f2ord(float f) {
-  const int i = __float_as_int(f);
-  return i >= 0 ? i : i ^ 0x7FFFFFFF;
-}
-__device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF); }
+constexpr int kTopkUnroll = 4;   // chunks a thread has in flight in the first pass
 
 // fp32 score error bound: a32 = z * (1/tau) and g32 from CUDA's logf / log1pf.
 __device__ __forceinline__ float score_err(float a32, float g32) {
@@ -52,15 +47,6 @@ struct TopkSmem {
   double s64[kTopkMax + 1];
   int i64[kTopkMax + 1];
 };
-
-template <typename TIn>
-__device__ __forceinline__ float ld_elem(const TIn* p, int i);
-template <>
-__device__ __forceinline__ float ld_elem<float>(const float* p, int i) { return p[i]; }
-template <>
-__device__ __forceinline__ float ld_elem<uint16_t>(const uint16_t* p, int i) {
-  return __uint_as_float((uint32_t)p[i] << 16);
-}
 
 // Inserts (s, d, v) into a descending list of length n held in a column of
 // shared memory (entry j at j * stride; ties to the lower v); returns the upper
@@ -164,136 +150,6 @@ __device__ __noinline__ void exact_topk_row(const TIn* row, int V, int k1, float
   }
 }
 
-// Eight consecutive entries of a row (one 16-byte chunk of bf16, two of fp32)
-// as floats; entries at or past V read as -inf.  `hint` is the L2 policy of
-// the vector loads.  The raw form (load8_raw, then unpack8) lets a thread keep
-// several chunks in flight.
-template <typename TIn>
-__device__ __forceinline__ void load8(const TIn* row, int v0, int V, bool vec, uint64_t hint,
-                                      float* z);
-template <>
-__device__ __forceinline__ void load8<uint16_t>(const uint16_t* row, int v0, int V, bool vec,
-                                                uint64_t hint, float* z) {
-  if (vec && v0 + 8 <= V) {
-    const uint4 u = ldg_hint(row + v0, hint);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      z[2 * j] = __uint_as_float(w[j] << 16);
-      z[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) z[j] = v0 + j < V ? ld_elem<uint16_t>(row, v0 + j) : -INFINITY;
-  }
-}
-template <>
-__device__ __forceinline__ void load8<float>(const float* row, int v0, int V, bool vec,
-                                             uint64_t hint, float* z) {
-  if (vec && v0 + 8 <= V) {
-    const uint4 a = ldg_hint(row + v0, hint), b = ldg_hint(row + v0 + 4, hint);
-    z[0] = __uint_as_float(a.x); z[1] = __uint_as_float(a.y);
-    z[2] = __uint_as_float(a.z); z[3] = __uint_as_float(a.w);
-    z[4] = __uint_as_float(b.x); z[5] = __uint_as_float(b.y);
-    z[6] = __uint_as_float(b.z); z[7] = __uint_as_float(b.w);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) z[j] = v0 + j < V ? row[v0 + j] : -INFINITY;
-  }
-}
-
-template <typename TIn>
-struct Raw8 {
-  uint4 a, b;  // bf16: a only
-};
-template <typename TIn>
-__device__ __forceinline__ Raw8<TIn> load8_raw(const TIn* row, int v0, int V, bool vec,
-                                               uint64_t hint) {
-  Raw8<TIn> r;
-  if (vec && v0 + 8 <= V) {
-    r.a = ldg_hint(row + v0, hint);
-    if (sizeof(TIn) == 4) r.b = ldg_hint(row + v0 + 4, hint);
-  } else {
-    float zz[8];
-    load8<TIn>(row, v0, V, false, hint, zz);
-    if (sizeof(TIn) == 2) {
-      uint32_t w[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        w[j] = (__float_as_uint(zz[2 * j]) >> 16) | (__float_as_uint(zz[2 * j + 1]) & 0xFFFF0000u);
-      r.a = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-      r.a = make_uint4(__float_as_uint(zz[0]), __float_as_uint(zz[1]), __float_as_uint(zz[2]),
-                       __float_as_uint(zz[3]));
-      r.b = make_uint4(__float_as_uint(zz[4]), __float_as_uint(zz[5]), __float_as_uint(zz[6]),
-                       __float_as_uint(zz[7]));
-    }
-  }
-  return r;
-}
-template <typename TIn>
-__device__ __forceinline__ void unpack8(const Raw8<TIn>& r, float* z) {
-  if (sizeof(TIn) == 2) {
-    const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      z[2 * j] = __uint_as_float(w[j] << 16);
-      z[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-  } else {
-    z[0] = __uint_as_float(r.a.x); z[1] = __uint_as_float(r.a.y);
-    z[2] = __uint_as_float(r.a.z); z[3] = __uint_as_float(r.a.w);
-    z[4] = __uint_as_float(r.b.x); z[5] = __uint_as_float(r.b.y);
-    z[6] = __uint_as_float(r.b.z); z[7] = __uint_as_float(r.b.w);
-  }
-}
-constexpr int kTopkUnroll = 4;   // chunks a thread has in flight in the first pass
-
-// The k-th largest of one value per thread of the CTA (-inf if fewer than k
-// are finite): k rounds of warp maxima, each removing one winning lane, then
-// the same over the warps' k best.
-__device__ __noinline__ float cta_kth_largest(float v, int k, float* buf /* [nwarps * k] */) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int r = 0; r < k; ++r) {
-    float w = v;
-    asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(w));
-    const unsigned hit = __ballot_sync(0xffffffffu, v == w && w > -INFINITY);
-    if (hit && lane == __ffs(hit) - 1) v = -INFINITY;
-    if (lane == 0) buf[warp * k + r] = hit ? w : -INFINITY;
-  }
-  __syncthreads();
-  float res = -INFINITY;
-  if (warp == 0) {
-    const int n = nw * k;  // <= 16 * 16: at most 8 per lane
-    float h[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) h[i] = lane + 32 * i < n ? buf[lane + 32 * i] : -INFINITY;
-    for (int r = 0; r < k; ++r) {
-      float m = h[0];
-#pragma unroll
-      for (int i = 1; i < 8; ++i) m = fmaxf(m, h[i]);
-      float w = m;
-      asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(w));
-      const unsigned hit = __ballot_sync(0xffffffffu, m == w && w > -INFINITY);
-      if (hit && lane == __ffs(hit) - 1) {
-        bool done = false;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (!done && h[i] == w) {
-            h[i] = -INFINITY;
-            done = true;
-          }
-      }
-      res = hit ? w : -INFINITY;
-    }
-    if (lane == 0) buf[0] = res;
-  }
-  __syncthreads();
-  res = buf[0];
-  __syncthreads();
-  return res;
-}
-
 // Dense rows.  A persistent CTA takes rows in turn and reads each twice:
 //   pass 1 (HBM, kept in L2 with an evict-last hint): the row's log-sum-exp
 //     (one exp2 per entry, online per thread) and each thread's largest logit;
@@ -351,7 +207,8 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_dense_kernel(
       unpack8<TIn>(raw[u], zz);
       float cm = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) cm = fmaxf(cm, zz[j]);
+      for (int j = 0; j < 8; ++j) cm = fmax_nan(cm, zz[j]);
+      bad |= cm != cm;  // a NaN, even one met while every earlier entry was -inf
       if (cm > zmax) {
         zmax = cm;
 #pragma unroll
@@ -371,7 +228,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_dense_kernel(
     }
     // lse: CTA combine of (m, S) in fp64
     // a NaN entry leaves S NaN (its exp2 is NaN), a +inf entry makes m +inf
-    bad = m == INFINITY || S != S;
+    bad = bad || m == INFINITY || S != S;
     float M = warp_max(m);
     float Sw = (m == -INFINITY) ? 0.f : S * ex2((m - M) * cT);
     Sw = warp_sum(Sw);

@@ -90,6 +90,25 @@ def test_host_argument_checks_need_no_gpu():
                            None, None) == lib.SD_ERR_INVALID_ARG    # unknown reward kind
     assert L.sd_metasd_ucb(None, 0, None, None, 0, 4, 2, 0, 2.0, None, None, None, None, None,
                            None) == lib.SD_OK                        # empty batch
+    assert L.ngram_table_bytes(1000, 10) == 0 and L.ngram_table_bytes(16, 10) == 0   # not 2^j >= 32
+    assert L.ngram_table_bytes(1024, 10) == 1024 * (8 + 4 + 80)
+    assert L.ngram_table_bytes(1024, 17) == 0
+    assert L.ngram_workspace_bytes(16385) == 0 and L.ngram_workspace_bytes(100) == 4 * 202
+    assert L.ngram_table_clear(vp(16), 1000, 10, None) == lib.SD_ERR_INVALID_ARG
+    assert L.ngram_store_update(vp(16), 1024, 10, vp(16), 4, vp(16), vp(16), 5, vp(16), 1 << 20,
+                                None, None) == lib.SD_ERR_INVALID_ARG   # n > 3
+    assert L.ngram_store_update(vp(16), 1024, 10, vp(16), 2, vp(16), vp(16), 5, vp(16), 40,
+                                None, None) == lib.SD_ERR_INVALID_ARG   # workspace too small
+    assert L.ngram_store_update(vp(16), 1024, 10, vp(16), 2, vp(16), vp(16), 20000, vp(16), 1 << 20,
+                                None, None) == lib.SD_ERR_UNSUPPORTED
+    assert L.ngram_store_update(vp(16), 1024, 10, None, 2, None, None, 0, None, 0, None,
+                                None) == lib.SD_OK                      # empty batch
+    assert L.ngram_store_lookup(vp(8), 1024, 10, vp(16), 2, 3, vp(16), vp(16), None, None,
+                                None) == lib.SD_ERR_INVALID_ARG         # table not 16-byte aligned
+    assert L.ngram_observe_topk(vp(16), 1, 4, 10, 10, None, 5, 10, 1.0, vp(16), vp(16), None,
+                                None) == lib.SD_ERR_INVALID_ARG         # U > rows without row_ids
+    assert L.ngram_observe_topk(vp(16), 1, 4, 10, 10, None, 4, 17, 1.0, vp(16), vp(16), None,
+                                None) == lib.SD_ERR_INVALID_ARG         # k > 16
     assert L.sd_draft_sample(vp(1), 1, 4, 10, 10, 1.0, 0, 0, 0xFFFFFFFE, vp(1), None, None,
                              None) == lib.SD_ERR_INVALID_ARG        # row ids past 2^32
     assert L.sd_draft_sample(None, 1, 0, 10, 10, 1.0, 0, 0, 0, None, None, None,

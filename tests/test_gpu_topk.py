@@ -144,3 +144,22 @@ def test_sparse_edge_cases():
     g, _ = run_sparse(ix[2:], pr[2:], 10, 0.5, 7, 3)     # k = L: a full permutation
     o = oracle.gumbel_topk_sparse(ix[2:], pr[2:], 10, 0.5, 7, 3)
     assert np.array_equal(g, o["idx"])
+
+
+def test_dense_nan_behind_masked_entries():
+    """A NaN met while every earlier entry of the thread's stream is -inf still
+    marks the row non-finite."""
+    rng = np.random.default_rng(12)
+    z = (rng.standard_normal((3, 20000)) * 2).astype(np.float32)
+    z[1, 0] = np.nan
+    z[1, 1:8] = -np.inf
+    z[2, 8 * 513] = np.nan          # second chunk of thread 1, first chunk all -inf
+    z[2, 8:16] = -np.inf
+    z[2, 8 * 513 + 1:8 * 514] = -np.inf
+    z = gen.bf16_bits_to_f32(gen.f32_to_bf16_bits(z))
+    g = run_dense(z, 4, 1.0, 2, 0)
+    o = oracle.gumbel_topk(z, 4, 1.0, 2, 0)
+    assert g["err"] == o["err"] == oracle.DEV_NONFINITE
+    assert np.all(g["idx"][1:] == -1)
+    compare_dense({k: v[:1] if k != "err" else 0 for k, v in g.items()},
+                  {**{k: v[:1] for k, v in o.items() if k not in ("err",)}, "err": 0}, "nanrow")

@@ -334,7 +334,9 @@ SMCSD_API sd_status sd_metasd_ucb(const float* tv, int64_t ld_tv, const int32_t*
  *   keys u64 [C] | counts i32 [C] | idx i32 [C][k] | prob f32 [C][k];
  * capacity C a power of two in [32, 2^40]; 1 <= k <= 16.  A key is the exact
  * n-gram (1 <= n <= 3 token ids in [0, 2^20)); slots are found by linear
- * probing from a hash of the key.  Nothing is ever deleted.
+ * probing from a hash of the key.  Nothing is ever deleted.  Which slot a new
+ * n-gram takes depends on the order in which concurrent claims land, so the
+ * buffer's bytes may differ between runs; every lookup result does not.
  */
 /* Bytes of a table of C slots with k entries each (0 if C or k is invalid). */
 SMCSD_API size_t ngram_table_bytes(int64_t capacity, int k);
@@ -382,6 +384,22 @@ SMCSD_API sd_status ngram_store_update(void* table, int64_t capacity, int k, con
                                        int n, const int32_t* idx, const float* prob, int U,
                                        void* workspace, size_t workspace_bytes, uint32_t* dev_err,
                                        void* stream);
+
+/*
+ * ngram_store_update_noalloc -- ngram_store_update without a caller
+ * workspace: the library's own fixed device array (room for 16384
+ * observations) serves as the workspace, and the call allocates nothing.
+ * The paper has no counterpart; it exists for callers that may not allocate
+ * device memory.  Nothing in the array must start at zero.  Every call
+ * shares the one array, so calls that overlap on the GPU (other streams,
+ * other host threads) race on it: keep them ordered.
+ * Arguments, requirements and faults as ngram_store_update; U > 16384 ->
+ * SD_ERR_UNSUPPORTED.
+ */
+SMCSD_API sd_status ngram_store_update_noalloc(void* table, int64_t capacity, int k,
+                                               const int32_t* ctx, int n, const int32_t* idx,
+                                               const float* prob, int U, uint32_t* dev_err,
+                                               void* stream);
 
 /*
  * ngram_store_lookup -- the stored rows of Q n-grams.

@@ -25,8 +25,8 @@ REWARD_BD, REWARD_BE = 0, 1
 EXPORTS = ("smcsd_score", "smcsd_resample", "smcsd_resample_adaptive", "kv_pagetable_remap",
            "sd_verify_reject", "gumbel_topk", "gumbel_topk_sparse", "sd_draft_sample",
            "sd_metasd_ucb", "ngram_table_clear", "ngram_observe_topk", "ngram_store_update",
-           "ngram_store_lookup", "ngram_table_bytes", "ngram_workspace_bytes", "sd_status_string",
-           "sd_version")
+           "ngram_store_lookup", "ngram_store_update_noalloc", "ngram_table_bytes",
+           "ngram_workspace_bytes", "sd_status_string", "sd_version")
 
 _lib = None
 
@@ -66,11 +66,12 @@ def load():
     L.ngram_store_update.argtypes = [vp, i64, i32, vp, i32, vp, vp, i32, vp, ctypes.c_size_t, vp,
                                      vp]
     L.ngram_store_lookup.argtypes = [vp, i64, i32, vp, i32, i32, vp, vp, vp, vp, vp]
+    L.ngram_store_update_noalloc.argtypes = [vp, i64, i32, vp, i32, vp, vp, i32, vp, vp]
     L.ngram_table_bytes.argtypes = [i64, i32]
     L.ngram_table_bytes.restype = ctypes.c_size_t
     L.ngram_workspace_bytes.argtypes = [i32]
     L.ngram_workspace_bytes.restype = ctypes.c_size_t
-    for name in EXPORTS[:13]:
+    for name in EXPORTS[:14]:
         getattr(L, name).restype = ctypes.c_int
     L.sd_status_string.argtypes = [ctypes.c_int]
     L.sd_status_string.restype = ctypes.c_char_p
@@ -361,6 +362,20 @@ def ngram_store_update(table, capacity, k, ctx, idx, prob, workspace, dev_err=No
                                    U, _p(workspace), workspace.numel(), _p(dev_err),
                                    _stream(stream))
     _check("ngram_store_update", st)
+
+
+def ngram_store_update_noalloc(table, capacity, k, ctx, idx, prob, dev_err=None, stream=None):
+    """ngram_store_update with the library's own workspace: allocates nothing.
+    Calls that overlap on the GPU race on that workspace."""
+    _table(table, capacity, k)
+    U, n = ctx.shape
+    _want(ctx, torch.int32, (U, n), "ctx")
+    _want(idx, torch.int32, (U, k), "idx")
+    _want(prob, torch.float32, (U, k), "prob")
+    _check_err(dev_err)
+    st = load().ngram_store_update_noalloc(_p(table), int(capacity), int(k), _p(ctx), n, _p(idx),
+                                           _p(prob), U, _p(dev_err), _stream(stream))
+    _check("ngram_store_update_noalloc", st)
 
 
 def ngram_store_lookup(table, capacity, k, ctx, idx_out, prob_out, count_out=None, dev_err=None,

@@ -657,3 +657,25 @@ extern "C" sd_status ngram_store_lookup(const void* table, int64_t capacity, int
       dev_err);
   return cudaGetLastError() == cudaSuccess ? SD_OK : SD_ERR_CUDA;
 }
+
+// ------------------------------------------------------------------ update without a workspace
+// The workspace of ngram_store_update taken from a fixed device array of this
+// library instead of the caller, for callers that must not allocate.  It holds
+// room for kUpdateMax observations; the sort writes every entry the merge
+// reads, so nothing in it must start at zero.  All calls share the one array:
+// calls that overlap on the GPU race on it.
+static __device__ __align__(256) int32_t g_ngram_scratch[2 * kUpdateMax + 2];
+
+extern "C" sd_status ngram_store_update_noalloc(void* table, int64_t capacity, int k,
+                                                const int32_t* ctx, int n, const int32_t* idx,
+                                                const float* prob, int U, uint32_t* dev_err,
+                                                void* stream) {
+  if (U > kUpdateMax) return SD_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (cudaGetSymbolAddress(&scratch, g_ngram_scratch) != cudaSuccess) {
+    cudaGetLastError();
+    return SD_ERR_CUDA;
+  }
+  return ngram_store_update(table, capacity, k, ctx, n, idx, prob, U, scratch,
+                            sizeof(g_ngram_scratch), dev_err, stream);
+}

@@ -451,7 +451,8 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
-PER_CONFIGS = ("smc_small", "smc_batch", "verify", "topk_dense", "topk_sparse")
+PER_CONFIGS = ("smc_small", "smc_batch", "verify", "topk_dense", "topk_sparse", "draft", "ngram",
+               "bandit")
 
 
 def per_config(args, hbm_peak, peak_kind):
@@ -590,6 +591,82 @@ def per_config(args, hbm_peak, peak_kind):
                                   {"config": {"rows": rows, "L": cfg.sparse_L, "k": k, "tau": cfg.tau,
                                               "l2": "flushed; hot_* without the flush"},
                                    "hot_ms_mean": hms, "hot_ms_median": hmed})
+        elif name == "draft":
+            # the draft step's sampler over every draft row of the smc_batch round
+            cfg = gen.CONFIGS["smc_batch"]
+            d = sdev.gen_config_device(cfg)
+            zD = d["zD"].reshape(-1, cfg.V)
+            rows = zD.shape[0]
+            toks = torch.empty((rows,), dtype=torch.int32, device=dev)
+            lq = torch.empty((rows,), dtype=torch.float32, device=dev)
+
+            def dr(i):
+                lib.sd_draft_sample(zD, cfg.tau, cfg.seed, i, toks, logq_out=lq, dev_err=err)
+            alg = rows * (cfg.V * 2 + 8)
+            ms, med, clocks = timed(dr, True, n)
+            out[name] = entry(ms, med, alg, rows, "rows_per_s", clocks,
+                              {"config": {"rows": rows, "V": cfg.V, "logits": cfg.dtype,
+                                          "tau": cfg.tau, "l2": "flushed",
+                                          "rows_from": "smc_batch draft tensor"}})
+            del d
+        elif name == "ngram":
+            # STAND store: 512 observed positions of a 152064-entry vocabulary,
+            # bigram contexts drawn Zipf(1.2) from 2048 n-grams, top-10 rows
+            import dataclasses
+            cfg = dataclasses.replace(gen.CONFIGS["topk"], B=512)
+            U, V, k, nn, cap = cfg.B, cfg.V, 10, 2, 1 << 16
+            z = sdev.gen_config_device(cfg)["z"]
+            rng = np.random.default_rng(cfg.seed)
+            pool = rng.integers(0, V, size=(2048, nn)).astype(np.int32)
+            ctx = torch.from_numpy(pool[np.minimum(rng.zipf(1.2, size=U) - 1, 2047)]).to(dev)
+            oi = torch.empty((U, k), dtype=torch.int32, device=dev)
+            op = torch.empty((U, k), dtype=torch.float32, device=dev)
+            tab = lib.NgramTable(cap, k, max_update=U)
+
+            def obs(i):
+                lib.ngram_observe_topk(z, k, cfg.tau, oi, op, dev_err=err)
+            alg_o = U * (V * 2 + k * 8)
+            ms, med, clocks = timed(obs, True, n)
+            out["ngram_observe"] = entry(ms, med, alg_o, U, "rows_per_s", clocks,
+                                         {"config": {"rows": U, "V": V, "k": k, "logits": cfg.dtype,
+                                                     "tau": cfg.tau, "l2": "flushed"}})
+
+            def upd(i):
+                tab.update(ctx, oi, op, dev_err=err)
+            # reads: contexts and rows; the rows of every touched n-gram read and written
+            alg_u = U * (nn * 4 + k * 8) + 2 * U * (8 + 4 + k * 8)
+            ms, med, clocks = timed(upd, False, n)
+            out["ngram_update"] = entry(ms, med, alg_u, U, "observations_per_s", clocks,
+                                        {"config": {"observations": U, "n": nn, "k": k,
+                                                    "capacity": cap, "distinct_ngrams": 2048,
+                                                    "l2": "hot (kilobyte-scale inputs)"}})
+            li = torch.empty((U, k), dtype=torch.int32, device=dev)
+            lp_ = torch.empty((U, k), dtype=torch.float32, device=dev)
+            cnt = torch.empty((U,), dtype=torch.int32, device=dev)
+
+            def look(i):
+                tab.lookup(ctx, li, lp_, count_out=cnt, dev_err=err)
+            alg_l = U * (nn * 4 + 8 + 4 + k * 8) + U * (k * 8 + 4)
+            ms, med, clocks = timed(look, False, n)
+            out["ngram_lookup"] = entry(ms, med, alg_l, U, "queries_per_s", clocks,
+                                        {"config": {"queries": U, "n": nn, "k": k, "capacity": cap,
+                                                    "l2": "hot (kilobyte-scale inputs)"}})
+            del z
+        elif name == "bandit":
+            # MetaSD-UCB round for 4096 sequences, 8 drafters, K = 5, BD reward
+            B, M, K = 4096, 8, 5
+            tvb = torch.rand((B, K), device=dev)
+            arm = torch.full((B,), -1, dtype=torch.int32, device=dev)
+            pulls = torch.zeros((B, M), dtype=torch.int32, device=dev)
+            sums = torch.zeros((B, M), dtype=torch.float64, device=dev)
+
+            def ban(i):
+                lib.sd_metasd_ucb(arm, pulls, sums, arm, K, tv=tvb, c=2.0, dev_err=err)
+            alg = B * (K * 4 + 4 + 4) + 2 * B * M * 12
+            ms, med, clocks = timed(ban, False, n)
+            out[name] = entry(ms, med, alg, B, "sequences_per_s", clocks,
+                              {"config": {"B": B, "M": M, "K": K, "reward": "BD",
+                                          "l2": "hot (kilobyte-scale inputs)"}})
         torch.cuda.empty_cache()
     return out
 

@@ -377,4 +377,26 @@ __device__ __forceinline__ void raise_err(uint32_t* dev_err, uint32_t bits) {
   if (dev_err) atomicOr(dev_err, bits);
 }
 
+// Bounded wait on an mbarrier phase, with a CTA-wide abort flag.  Gives up
+// after limit_ns of polling (the clock and the flag are read every 16th
+// poll), then sets the flag and records SD_DEV_TIMEOUT | site.  An abortable
+// wait also returns at once, without an error of its own, when another wait
+// of the CTA has already given up; a non-abortable one (a wait that orders a
+// bulk copy into shared memory) keeps waiting for its phase up to its own limit.
+__device__ __forceinline__ void bounded_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             uint32_t* err, uint32_t site, bool abortable,
+                                             uint64_t limit_ns = kWaitNs) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if ((i & 15u) == 0) {
+      if (abortable && *abort_flag) return;
+      if (globaltimer_ns() - t0 >= limit_ns) break;
+    }
+    if (mbar_try_wait(bar, parity)) return;
+  }
+  *abort_flag = 1;
+  raise_err(err, SD_DEV_TIMEOUT | site);
+}
+
 }  // namespace smcsd

@@ -78,25 +78,15 @@ enum WaitSite : uint32_t {
   kWsAdone = 1u << 13, kWsBook = 1u << 14, kWsBmsg = 1u << 15
 };
 
-// Bounded wait (kWaitNs of polling).  After one expiry every later abortable
-// wait of the CTA returns at once (outputs are then garbage, SD_DEV_TIMEOUT is
-// set, nothing hangs).  The waits that order the bulk copies into the ring are
-// not abortable: a stage is refilled only after every producer has seen its
-// last copy land, so no copy can still be in flight into a CTA that finishes.
+// Bounded waits (common.cuh: bounded_wait, kWaitNs of polling).  After one
+// expiry every later abortable wait of the CTA returns at once (outputs are
+// then garbage, SD_DEV_TIMEOUT is set, nothing hangs).  The waits that order
+// the bulk copies into the ring are not abortable: a stage is refilled only
+// after every producer has seen its last copy land, so no copy can still be
+// in flight into a CTA that finishes.
 __device__ __forceinline__ void swait(uint64_t* bar, uint32_t parity, SmcTail* tl, uint32_t* err,
                                       uint32_t site, bool abortable = true) {
-  if (mbar_try_wait(bar, parity)) return;
-  volatile int* ab = &tl->abort_flag;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if ((i & 15u) == 0) {  // (the abort flag and the clock every 16 polls only)
-      if (abortable && *ab) return;
-      if (globaltimer_ns() - t0 >= kWaitNs) break;
-    }
-    if (mbar_try_wait(bar, parity)) return;
-  }
-  *ab = 1;
-  raise_err(err, SD_DEV_TIMEOUT | site);
+  bounded_wait(bar, parity, &tl->abort_flag, err, site, abortable);
 }
 
 // fp64 lse of a row's target and draft halves from the C slice partials of its

@@ -144,7 +144,8 @@ def test_testing_library_exports_its_probes():
     assert os.path.exists(tl), "build the libraries first (__graft_entry__.build())"
     names = subprocess.run(["nm", "-D", "--defined-only", tl], capture_output=True, text=True,
                            check=True).stdout
-    assert "smcsd_testing_philox" in names and "smcsd_testing_stream" in names
+    syms = {line.split()[-1] for line in names.splitlines() if line.strip()}
+    assert {"smcsd_testing_philox", "smcsd_testing_stream", "smcsd_testing_wait"} <= syms
     main = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
                           text=True, check=True).stdout
     assert "smcsd_testing" not in main

@@ -11,21 +11,24 @@ Definitions followed (all readings are listed in the project's design notes):
     scores draft token x_{k+1}.  The bonus token is drawn from p_T, so its ratio
     is 1 and it does not enter the weight.
   * same page, section 2 (bonus token): each round also commits one token drawn
-    from the target at position K+1.  Reading: Gumbel-max,
-        bonus = argmax_v ( z_T[K, v] / tau + g_v ),  g_v ~ Gumbel(0, 1)
-    with g_v from Philox stream 1, row id = b * N + n; ties go to the lower v.
+    from the target at position K+1.  Reading: the exact two-level Gumbel-max
+    of ``oracle.blockdraw`` over a = z_T[K] / tau, block noise from Philox
+    stream 9 and entry noise from stream 1, row id = b * N + n (for V <= 128:
+    bonus = argmax_v (a_v + g_v), g_v from stream 1; ties to the lower v).
   * METASD page, section 2 (Block Divergence built on total-variation
     distance): per row, tv = 1/2 * sum_v | p_T(v) - q_D(v) |, reported at all
     K+1 positions.
 
 Parity status: lse / lp / logw / tv are the fp64 definition written out and are
 pinned by closed forms and invariants (tests/test_oracle_score.py).  The bonus
-token is pinned by a chi-square test of Gumbel-max against softmax at V = 16.
+token is pinned by a chi-square test of Gumbel-max against softmax at V = 16
+and by the two-level draw's own pins (tests/test_oracle_blockdraw.py).
 """
 
 import numpy as np
 
-from .philox import STREAM_BONUS, gumbel_from_uniform, stream_words, uniform_from_bits
+from .blockdraw import block_gumbel_argmax
+from .philox import STREAM_BONUS, STREAM_BONUS_BLOCK, gumbel_from_uniform, stream_words, uniform_from_bits
 
 # Device error-word bits (the library's caller-visible error word uses the same values).
 DEV_TOKEN_OOB = 1
@@ -149,8 +152,8 @@ def smcsd_score(zT, zD, draft_tokens, tau, seed, rnd, logw_prev=None, b0=0, log_
             logw[b, n] = acc
             tokens[b, n, :K] = draft_tokens[b, n]
             if not np.isnan(lse_t[K]):
-                g = bonus_noise(seed, rnd, (b0 + b) * N + n, V)
-                idx, mg = gumbel_argmax(a[K] + g)
+                idx, mg = block_gumbel_argmax(a[K], seed, rnd, STREAM_BONUS_BLOCK, STREAM_BONUS,
+                                              (b0 + b) * N + n)
                 bonus[b, n] = idx
                 margin[b, n] = mg
             tokens[b, n, K] = bonus[b, n]

@@ -89,6 +89,7 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_STREAM_TOPK_DENSE 5u
 #define SD_STREAM_TOPK_SPARSE 6u
 #define SD_STREAM_DRAFT 8u
+#define SD_STREAM_BONUS_BLOCK 9u
 
 /*
  * smcsd_score -- scoring step of one SMC-SD round ([SMC-SD] section 2, scoring
@@ -101,8 +102,13 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
  *   logw[b,n] = logw_prev[b,n] + phi[b,n] + sum_{k<K} (lp - lq)
  *                                                         (importance weight);
  *   tv[b,n,k] = 1/2 sum_v |p_v - q_v| at all K+1 rows    (block divergence);
- *   bonus[b,n] = argmax_v (zT[b,n,K,v]/tau + g_v), g from stream 1 with row
- *                id b*N+n, ties to the lower v           (bonus token).
+ *   bonus[b,n] = a sample of softmax(zT[b,n,K,:]/tau) by an exact two-level
+ *                Gumbel-max over blocks of 128 entries: block
+ *                j* = argmax_j (log sum_{v in j} e^{z_v/tau} + G_j), G from
+ *                stream 9, then v* = argmax_{v in j*} (z_v/tau + g_v), g from
+ *                stream 1 (both: row id b*N+n, counter entry j or v; ties to
+ *                the lower index).  V <= 128: plain Gumbel-max on stream 1.
+ *                                                        (bonus token)
  *
  * zT, zD        device, [B, N, K+1, V] at row stride ld, dtype dt (fp32 or
  *               bf16).  Both tensors have K+1 rows per particle.

@@ -57,7 +57,7 @@ struct alignas(16) Msg {
 // best's lower bound the winner is exact; otherwise it is settled in fp64.
 struct Cand {
   float s, lo, hi, ohi;
-  int idx, pad0, pad1, pad2;
+  int idx, aux, pad1, pad2;  // aux: a value that travels with the candidate (-1: none)
 };
 
 struct Cand64 {
@@ -72,7 +72,8 @@ __device__ __forceinline__ Cand cand_empty() {
   c.hi = -INFINITY;
   c.ohi = -INFINITY;
   c.idx = 0x7FFFFFFF;
-  c.pad0 = c.pad1 = c.pad2 = 0;
+  c.aux = -1;
+  c.pad1 = c.pad2 = 0;
   return c;
 }
 __device__ __forceinline__ Cand cand_merge(const Cand& a, const Cand& b) {
@@ -89,7 +90,8 @@ __device__ __forceinline__ Cand cand_shfl(const Cand& c, int o) {
   r.hi = __shfl_xor_sync(0xffffffffu, c.hi, o);
   r.ohi = __shfl_xor_sync(0xffffffffu, c.ohi, o);
   r.idx = __shfl_xor_sync(0xffffffffu, c.idx, o);
-  r.pad0 = r.pad1 = r.pad2 = 0;
+  r.aux = __shfl_xor_sync(0xffffffffu, c.aux, o);
+  r.pad1 = r.pad2 = 0;
   return r;
 }
 __device__ __forceinline__ Cand warp_cand(Cand c) {
@@ -128,7 +130,8 @@ static __device__ __noinline__ Cand bonus_cand_a(float a32, float u, int v) {
   cd.hi = cd.s + d;
   cd.ohi = -INFINITY;
   cd.idx = v;
-  cd.pad0 = cd.pad1 = cd.pad2 = 0;
+  cd.aux = -1;
+  cd.pad1 = cd.pad2 = 0;
   return cd;
 }
 

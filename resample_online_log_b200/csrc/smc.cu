@@ -17,9 +17,11 @@ namespace smcsd {
 //   producers (one per 32 x 32 entries of the slice), row by row: move the
 //     row's slices from the ring to registers, warp maxima, exps (one MUFU
 //     exp2 per entry) and sums; the exps of both halves go to tensor memory
-//     (TMEM, two row buffers per warp); post the (max, sum) partials.  In the
-//     row after a particle's last row they also screen that row's bonus-token
-//     candidates from its exps, still in TMEM.
+//     (TMEM, two row buffers per warp); post the (max, sum) partials.
+//     On a particle's last row they also sum the target exps of each
+//     128-entry block and post the best block candidate of the bonus draw
+//     (a two-level Gumbel-max: the block by log-mass plus block noise, then
+//     the entry inside it).
 //   consumers (four, one per TMEM lane quarter), one row behind: once the
 //     row's messages are in, rebuild its normalisers, read the exps back from
 //     TMEM and take the TV partial sum |p - q|; then hand the row buffer back.
@@ -29,13 +31,15 @@ namespace smcsd {
 //     the row path), sends each row's TV partial and bonus candidate to the
 //     leader, and refills the ring with bulk async copies (no multicast).
 //   bookkeeping (leader only): fp64 lse, log-probs, log-weights, TV and bonus
-//     tokens (near-ties settled exactly in fp64).
+//     tokens: the block from the candidates (a near-tie in fp64 over the
+//     row's blocks), then the entry inside it from its 128 logits.
 // MUFU work (producers) and the exchange plus TV (consumers) overlap; every
 // element is read from HBM once and exponentiated once.
 
 constexpr int kRing = 8;     // message slots per CTA
 constexpr int kLead = 2;     // rows a CTA's messages can run ahead of the leader's
 constexpr int kMaxStages = 4;
+constexpr int kBlk = 128;    // entries per block of the two-level bonus draw
 constexpr uint32_t kTmemCols = 512;  // all of the SM's tensor memory (one CTA per SM)
 constexpr int kConsumers = 4;        // phase-B warps, one per TMEM lane quarter
 constexpr int kMaxThreadsSmc = 640;  // up to 14 producers + 4 consumers + 2 service warps
@@ -55,7 +59,6 @@ struct alignas(128) SmcTail {
   uint64_t afull[2];  // producers done with a row (exps in TMEM, partials posted)
   uint64_t bfull[2];  // consumers done with a row (TV partials, candidates posted)
   uint64_t tfree[2];  // consumers done reading a TMEM row buffer
-  uint64_t sfin;      // producers posted the last row's bonus candidates
   uint64_t rbar[kRing], bbar[kRing], adone[kRing];
   int abort_flag;
   uint32_t tmem_base;
@@ -63,7 +66,7 @@ struct alignas(128) SmcTail {
   BMsg brecv[kRing][kMaxCluster];
   float4 wpart[2][kMaxWarps];
   float wtv[2][kConsumers];
-  Cand wcand[4][kMaxWarps];  // producers' bonus candidates, by row & 3
+  Cand wcand[4][kMaxWarps];  // producers' best bonus blocks, by row & 3
   // Raw logits of a row's draft token at its owner, by row & 3: producer warps
   // are not ordered among themselves, so the owner may post row it+2's value
   // before the slowest warp has finished row it (and so before the
@@ -128,29 +131,62 @@ __device__ __forceinline__ Norm row_norm(float pm1, float ps1, float pm2, float 
   return n;
 }
 
-// Exact fp64 bonus draw over a whole target row (a near-tie the fp32 screen
-// could not settle; rare).  One warp.
+// Exact steps of the bonus draw, a two-level Gumbel-max over blocks of kBlk
+// entries (the block by its log-mass plus block noise, then the entry inside
+// it by plain Gumbel-max).  One warp each; both are fallbacks for the rare
+// rows whose fp32 bounds do not settle a step.
+//
+// The block over a whole target row: lambda_j = log sum exp(z/tau), in fp64.
 template <typename TIn>
-__device__ __noinline__ int exact_bonus_row(const TIn* row, int V, double tau64, float inv_tau,
-                                            float lo_star, const Stream st, uint32_t rowid) {
+__device__ __noinline__ int exact_block_row(const TIn* row, int V, double tau64, const Stream st,
+                                            uint32_t rowid) {
   const int lane = threadIdx.x & 31;
+  const int nb = (V + kBlk - 1) / kBlk;
   double best = -INFINITY;
   int bi = 0x7FFFFFFF;
-  for (int q = lane; q * 4 < V; q += 32) {
-    const U4 w = st.at((uint32_t)q, rowid);
-    for (int j = 0; j < 4; ++j) {
-      const int v = q * 4 + j;
-      if (v >= V) break;
-      const float z = Elem<TIn>::get(row, v);
-      const float a32 = z * inv_tau;
-      if (!(a32 + kGumbelMaxF + 1e-3f >= lo_star)) continue;
-      const float g32 = gumbel_f32(uniform_f32(word_of(w, j)));
-      const float hi = a32 + g32 + 4e-6f + 4.8e-7f * (fabsf(a32) + 2.f * fabsf(g32));
-      if (!(hi >= lo_star)) continue;
-      const double s64 = (double)z / tau64 + gumbel_f64(uniform_f64(word_of(w, j)));
-      c64_merge(best, bi, s64, v);
-    }
+  for (int j = lane; j < nb; j += 32) {
+    const int v0 = j * kBlk, v1 = min(v0 + kBlk, V);
+    double m = -INFINITY;
+    for (int v = v0; v < v1; ++v) m = fmax(m, (double)Elem<TIn>::get(row, v) / tau64);
+    if (!(m > -INFINITY)) continue;
+    double sum = 0.0;
+    for (int v = v0; v < v1; ++v) sum += exp((double)Elem<TIn>::get(row, v) / tau64 - m);
+    const U4 w = st.at((uint32_t)(j >> 2), rowid);
+    c64_merge(best, bi, m + log(sum) + gumbel_f64(uniform_f64(word_of(w, j & 3))), j);
   }
+  warp_c64(best, bi);
+  return bi == 0x7FFFFFFF ? -1 : bi;
+}
+
+// The entry inside block j: argmax (z/tau + g_v), g from the entry stream at
+// the global position v (four entries, one Philox block, per lane); fp32
+// bounds first, fp64 if two entries come within them.
+template <typename TIn>
+__device__ __noinline__ int exact_in_block(const TIn* row, int V, int j, float inv_tau,
+                                           double tau64, const Stream st, uint32_t rowid) {
+  const int lane = threadIdx.x & 31;
+  const int v0 = j * kBlk + 4 * lane;
+  float z[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  U4 w = U4{0u, 0u, 0u, 0u};
+  Cand cd = cand_empty();
+  if (lane < kBlk / 4 && v0 < V) {
+    w = st.at((uint32_t)(v0 >> 2), rowid);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) z[t] = v0 + t < V ? Elem<TIn>::get(row, v0 + t) : -INFINITY;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (z[t] > -INFINITY)
+        cd = cand_merge(cd, bonus_cand_a(z[t] * inv_tau, uniform_f32(word_of(w, t)), v0 + t));
+  }
+  cd = warp_cand(cd);
+  if (cd.idx == 0x7FFFFFFF) return -1;
+  if (cd.ohi < cd.lo) return cd.idx;
+  double best = -INFINITY;
+  int bi = 0x7FFFFFFF;
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+    if (z[t] > -INFINITY)
+      c64_merge(best, bi, (double)z[t] / tau64 + gumbel_f64(uniform_f64(word_of(w, t))), v0 + t);
   warp_c64(best, bi);
   return bi == 0x7FFFFFFF ? -1 : bi;
 }
@@ -232,64 +268,12 @@ __device__ __forceinline__ uint4 load_chunk(const TIn* st, const TIn* g, int e0,
   return Chunk<TIn>::gather(st, g, e0, len, tma_len);
 }
 
-// Bonus-token screen over this thread's target entries of a particle's last
-// row, from the exps held in TMEM (relative to the warp max), in two halves of
-// sixteen entries (one loop body, kept small for the instruction cache): the
-// four Philox blocks of a half are drawn together (independent, so they
-// overlap); an entry whose y = e * rho = e^{a - Tref} proves it cannot win is
-// dropped before any log; the few kept entries become candidates with fp32
-// bounds, their logit over tau recovered as a = m/tau + ln(e) (m: the warp max
-// the exp is relative to; the error is far inside the candidate bounds).
-template <typename TIn>
-__device__ __forceinline__ Cand bonus_screen(uint32_t tcolT, int s0, int len, int tid, int ncomp,
-                                             float rho, float mw_a, const Stream bst,
-                                             uint32_t rowid) {
-  constexpr int EPC = Chunk<TIn>::EPC;
-  Cand cd = cand_empty();
-#pragma unroll 1
-  for (int h = 0; h < 2; ++h) {
-    float e[16];
-    __syncwarp();
-    tmem_ld16(tcolT + 16u * (uint32_t)h, e);
-    tmem_wait_ld();
-    // One bound for the half: with y <= ymax = emax * rho, keep_bonus needs
-    // u >= thr(ymax) (same fp32 steps, monotone), so a word whose top 23 bits
-    // m = w >> 9 fall below mstar fails for every entry here;
-    // u = (m + 1/2) 2^-23 >= thr  <=>  m >= thr 2^23 - 1/2 (exact in fp32).
-    float emax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) emax = fmaxf(emax, e[i]);
-    const float thr = (1.0f - (emax * rho) * 1.001f) - 2.4e-7f;
-    const uint32_t mstar = thr > 0.f ? (uint32_t)ceilf(thr * 8388608.f - 0.5f) : 0u;
-    U4 w[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {  // entries 16h + 4q .. +3 of this thread: one Philox block
-      const int i = 16 * h + 4 * q;
-      const int eg = (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
-      w[q] = bst.at((uint32_t)((s0 + eg) >> 2), rowid);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = 16 * h + 4 * q;
-      const int eg = (tid + (i / EPC) * ncomp) * EPC + (i % EPC);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if ((word_of(w[q], j) >> 9) < mstar) continue;
-        const float ej = e[4 * q + j];
-        const float u = uniform_f32(word_of(w[q], j));
-        if (keep_bonus(ej * rho, u) && eg + j < len && ej > 0.f)
-          cd = cand_merge(cd, bonus_cand_a(mw_a + logf(ej), u, s0 + eg + j));
-      }
-    }
-  }
-  return cd;
-}
-
 template <typename TIn>
 __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32_t cid, uint32_t G,
                              int nrows, bool want_tv) {
   const int lane = threadIdx.x & 31;
   const Stream bst(a.seed, a.round, SD_STREAM_BONUS);
+  const Stream blkst(a.seed, a.round, SD_STREAM_BONUS_BLOCK);
   const bool lane_tokens = a.K <= 32;
   double logw_acc = 0.0;
   bool unit_bad = false;
@@ -399,12 +383,16 @@ __device__ void smc_bookkeep(const ScoreArgs& a, SmcTail* tl, uint32_t C, uint32
       if (want_tv && lane == 0) a.tv_out[punit * a.R + pk] = prev_bad ? NAN : 0.5f * tv;
       if (pk == a.K) {
         c = warp_cand(c);
-        int winner;
-        if (prev_badT || c.idx == 0x7FFFFFFF) winner = -1;
-        else if (c.ohi < c.lo) winner = c.idx;
-        else
-          winner = exact_bonus_row<TIn>((const TIn*)a.zT + (punit * a.R + pk) * a.ld, a.V, a.tau64,
-                                        a.inv_tau, c.lo, bst, (uint32_t)punit);
+        // the block from the candidates when their bounds settle it (else in
+        // fp64 over the row), then the entry inside it from its 128 logits
+        int winner = -1;
+        if (!prev_badT && c.idx != 0x7FFFFFFF) {
+          const TIn* brow = (const TIn*)a.zT + (punit * a.R + pk) * a.ld;
+          const int jb = c.ohi < c.lo ? c.idx
+                                      : exact_block_row<TIn>(brow, a.V, a.tau64, blkst, (uint32_t)punit);
+          if (jb >= 0)
+            winner = exact_in_block<TIn>(brow, a.V, jb, a.inv_tau, a.tau64, bst, (uint32_t)punit);
+        }
         if (lane == 0) {
           a.bonus_out[punit] = winner;
           if (a.tokens_out) a.tokens_out[punit * a.R + a.K] = winner;
@@ -459,7 +447,6 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       mbar_init(&tl->bfull[b], kConsumers);
       mbar_init(&tl->tfree[b], kConsumers);
     }
-    mbar_init(&tl->sfin, (uint32_t)nA);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&tl->rbar[i], 1);
       mbar_init(&tl->bbar[i], 1);
@@ -539,8 +526,7 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
         tv = warp_sum(tv);
         const int pk = k == 0 ? a.R - 1 : k - 1;
         Cand cd = cand_empty();
-        if (pk == a.K) {  // the producers screened it during the next row (the last: on its own)
-          if (p == nrows - 1) swait(&tl->sfin, 0u, tl, a.dev_err, kWsBfull);
+        if (pk == a.K) {  // the producers posted its bonus blocks with the row
           if (lane < nA) cd = tl->wcand[p & 3][lane];
           cd = warp_cand(cd);
         }
@@ -649,30 +635,7 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
   int stage = 0;
   uint32_t phase = 0;
   int x_next = (nrows > 0 && a.K > 0) ? a.draft[(int64_t)cid * a.K] : -1;
-  float mwT_prev = -INFINITY;  // this warp's raw target max of the previous row
-
-  // Bonus-token screen of row p (a particle's last row) over this warp's entries,
-  // from its exps still in TMEM, once the row's messages give its max M.
-  auto screen = [&](int p, int64_t punit) {
-    swait(&tl->rbar[p % kRing], (uint32_t)((p / kRing) & 1), tl, a.dev_err, kWsRow);
-    __syncwarp();
-    const Msg* rv = tl->recv[p % kRing];
-    const bool has = lane < (int)C;
-    const Norm nm = row_norm(has ? rv[lane].mT : -INFINITY, has ? rv[lane].sT : 0.f,
-                             has ? rv[lane].mD : -INFINITY, has ? rv[lane].sD : 0.f, cT);
-    Cand cd = cand_empty();
-    if (!nm.badT && mwT_prev > -INFINITY) {
-      // Tref = M/tau + g_min - margin bounds the winning score from below
-      const float margin = 1e-5f + 2e-7f * fabsf(nm.MT * a.inv_tau);
-      const float rho = ex2((mwT_prev - nm.MT) * cT + (-kGumbelMinF + margin) * kLog2e);
-      cd = bonus_screen<TIn>(tcol + 64u * (uint32_t)(p & 1), s0, len, tid, ncomp, rho,
-                             mwT_prev * a.inv_tau, Stream(a.seed, a.round, SD_STREAM_BONUS),
-                             (uint32_t)punit);
-    }
-    cd = warp_cand(cd);
-    if (lane == 0) tl->wcand[p & 3][warp] = cd;
-  };
-
+  const Stream blkst(a.seed, a.round, SD_STREAM_BONUS_BLOCK);
   for (int it = 0; it < nrows; ++it) {
     const int x = k < a.K ? x_next : -1;
     {  // prefetch the draft token of row it+1
@@ -729,8 +692,11 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
     const uint32_t tb = tcol + 64u * (uint32_t)(it & 1);
     float2 accT = f2(0.f), accD = f2(0.f);
     float eT[8], eD[8];
+    const bool brow = k == a.K;  // a particle's last row: the bonus draw's block sums too
+    float bsum = 0.f;            // lane q < 8: the target exp sum of this warp's block q
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
+      float2 bacc = f2(0.f), dacc = f2(0.f);  // this chunk's sums (same order for both halves)
       uint4 vT, vD;
       if (HOLD) {
         vT = rT[HOLD ? c : 0];
@@ -749,8 +715,8 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
         eT[i + 1] = ex2(tT.y);
         eD[i] = ex2(tD.x);
         eD[i + 1] = ex2(tD.y);
-        accT = __fadd2_rn(accT, make_float2(eT[i], eT[i + 1]));
-        accD = __fadd2_rn(accD, make_float2(eD[i], eD[i + 1]));
+        bacc = __fadd2_rn(bacc, make_float2(eT[i], eT[i + 1]));
+        dacc = __fadd2_rn(dacc, make_float2(eD[i], eD[i + 1]));
         if (i + 2 == 8) {  // eight entries done: park them (whole warp, converged)
           const uint32_t col = (uint32_t)((c * EPC + j + 2) - 8);
           __syncwarp();
@@ -758,6 +724,49 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
           tmem_st8(tb + 32u + col, eD);
         }
       }
+      accT = __fadd2_rn(accT, bacc);
+      accD = __fadd2_rn(accD, dacc);
+      if (brow) {  // a chunk row of the warp is one block (fp32) or two (bf16: half-warps)
+        float sb = bacc.x + bacc.y;
+        if (EPC == 8) {
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) sb += __shfl_xor_sync(0xffffffffu, sb, o);
+          const float t0 = __shfl_sync(0xffffffffu, sb, 0), t1 = __shfl_sync(0xffffffffu, sb, 16);
+          if (lane == 2 * c) bsum = t0;
+          if (lane == 2 * c + 1) bsum = t1;
+        } else {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sb += __shfl_xor_sync(0xffffffffu, sb, o);
+          if (lane == c) bsum = sb;
+        }
+      }
+    }
+    if (brow) {
+      // Block candidates of the bonus draw: lambda_j = ln(sum) + m/tau (the exps
+      // are relative to the warp max m) plus the block's Gumbel noise, with fp32
+      // error bounds.  A block whose exps all flushed to 0 lies > 80 nats below
+      // this warp's best block and cannot win (block noise spans < 20).
+      Cand cd = cand_empty();
+      if (lane < 8 && bsum > 0.f) {
+        const int local = EPC == 8 ? (32 * warp + 16 * (lane & 1) + (lane >> 1) * ncomp) * 8
+                                   : (32 * warp + lane * ncomp) * 4;
+        if (local < len) {
+          const int jb = (s0 + local) / kBlk;
+          const U4 w = blkst.at((uint32_t)(jb >> 2), (uint32_t)unit);
+          const float g32 = gumbel_f32(uniform_f32(word_of(w, jb & 3)));
+          const float lam = logf(bsum) + mwTs * a.inv_tau;
+          const float sc = lam + g32;
+          // ln(sum) error: exp arguments rounded in fp32 (|t| <= 130 before
+          // flushing; the max term 2^-24 |m c| each), ex2.approx, the sum
+          const float d = score_err(lam, g32) + 2e-5f + 2e-7f * fabsf(mwTs * cT);
+          cd.s = sc;
+          cd.lo = sc - d;
+          cd.hi = sc + d;
+          cd.idx = jb;
+        }
+      }
+      cd = warp_cand(cd);
+      if (lane == 0) tl->wcand[it & 3][warp] = cd;
     }
     if (!HOLD) {  // pass 2 re-read the stage
       __syncwarp();
@@ -766,8 +775,6 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
     float sTw = accT.x + accT.y, sDw = accD.x + accD.y;
     warp_sum2(sTw, sDw);
     if (lane == 0) tl->wpart[it & 1][warp] = make_float4(mwT, sTw, mwD, sDw);
-    if (k == 0 && it > 0) screen(it - 1, unit - G);  // the previous row ended a particle
-    mwT_prev = mwT;
     __syncwarp();
     tmem_wait_st();
     tmem_fence_before();
@@ -780,11 +787,6 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       k = 0;
       unit += G;
     }
-  }
-  if (nrows > 0) {  // the last row ends a particle too
-    screen(nrows - 1, unit - G);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&tl->sfin);
   }
   __syncwarp();
   tmem_fence_before();
@@ -818,7 +820,8 @@ static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, Launc
   bool found = false;
   int64_t best_score = -1;
   for (int C = 1; C <= kMaxCluster; ++C) {
-    const int slice = (int)(((int64_t)(V + C - 1) / C + 7) / 8 * 8);
+    const int slice = (int)(((int64_t)(V + C - 1) / C + kBlk - 1) / kBlk * kBlk);  // whole blocks
+    if (C > 1 && (int64_t)(C - 1) * slice >= V) continue;  // no empty slice
     const int ncomp = std::max(32, (int)(((slice + kEPT - 1) / kEPT + 31) / 32 * 32));
     const int threads = ncomp + 32 * (kConsumers + 2);  // + consumers, communication, bookkeeping
     if (threads > kMaxThreadsSmc || ncomp / 32 > kMaxWarps) continue;

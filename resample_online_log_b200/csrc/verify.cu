@@ -394,7 +394,8 @@ __global__ void __launch_bounds__(kVThreads, 1) verify_rows_kernel(const VerifyA
           cd.lo = r4[e] - eb4[e] > 0.f ? logf(r4[e] - eb4[e]) + g32 - d : -INFINITY;
           cd.ohi = -INFINITY;
           cd.idx = v0 + e;
-          cd.pad0 = cd.pad1 = cd.pad2 = 0;
+          cd.aux = -1;
+          cd.pad1 = cd.pad2 = 0;
           best = cand_merge(best, cd);
           if (cd.lo > Tr) {
             Tr = cd.lo;

@@ -1,4 +1,4 @@
-"""Pins for the oracle's draft-step sampler (Gumbel-max over zD / tau)."""
+"""Pins for the oracle's draft-step sampler (two-level Gumbel-max over zD / tau)."""
 
 import numpy as np
 from scipy import special, stats
@@ -51,3 +51,18 @@ def test_masked_entries_never_drawn_and_bad_rows():
     frac7 = np.mean(x == 7)
     p7 = np.exp(0.5) / (1 + np.exp(0.5))
     assert abs(frac7 - p7) < 4 * np.sqrt(p7 * (1 - p7) / 20000)
+
+
+def test_draw_frequencies_match_softmax_v1000_blocks():
+    """V = 1000 (8 blocks of the two-level draw): 12000 rows against softmax, 20 bins."""
+    V, M = 1000, 12000
+    v = np.arange(V)
+    z = 2.0 * np.sin(v / 53.0) + np.cos(v / 7.0)
+    t = np.float64(np.float32(0.8))
+    p = np.exp(z / t - special.logsumexp(z / t))
+    x = oracle.sd_draft_sample(np.broadcast_to(z, (M, V)), 0.8, 4, 6)["tokens"]
+    bins = v // 50
+    counts = np.bincount(bins[x], minlength=20)
+    expect = np.bincount(bins, weights=p, minlength=20) * M
+    _, pval = stats.chisquare(counts, expect)
+    assert pval > 1e-3, pval

@@ -90,6 +90,7 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_STREAM_TOPK_SPARSE 6u
 #define SD_STREAM_DRAFT 8u
 #define SD_STREAM_BONUS_BLOCK 9u
+#define SD_STREAM_DRAFT_BLOCK 10u
 
 /*
  * smcsd_score -- scoring step of one SMC-SD round ([SMC-SD] section 2, scoring
@@ -265,9 +266,12 @@ SMCSD_API sd_status gumbel_topk_sparse(const int32_t* idx, const float* prob, in
  * from the drafter's own distribution ([SMC-SD] section 2: the draft model
  * extends each particle by K tokens, one position at a time; [STAND]
  * Methodology item 1: stochastic drafting samples the distribution instead of
- * taking its argmax).  Gumbel-max, exact:
- *   tokens[r] = argmax_v (zD[r, v] / tau + g_v), g from stream 8 with row id
- *               row0 + r, ties to the lower v;
+ * taking its argmax).  Exact two-level Gumbel-max over blocks of 128 entries:
+ *   block j*  = argmax_j (log sum_{v in j} e^{zD[r,v]/tau} + G_j), G from
+ *               stream 10;
+ *   tokens[r] = argmax_{v in j*} (zD[r, v] / tau + g_v), g from stream 8
+ *               (both: row id row0 + r, counter entry j or v, ties to the
+ *               lower index; V <= 128: plain Gumbel-max on stream 8);
  *   logq[r]   = zD[r, tokens[r]] / tau - logsumexp_v(zD[r, v] / tau),
  * the log q_D(x) an SMC-SD importance weight uses.  One call per draft
  * position: rows are all particles of all sequences at that position.

@@ -7,7 +7,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = ["abi.cu", "smc.cu", "verify.cu", "resample.cu", "pagetable.cu", "topk.cu",
-           "bandit.cu", "ngram.cu"]
+           "bandit.cu", "ngram.cu", "draft.cu"]
 LIB = os.path.join(HERE, "libsmcsd.so")
 TESTING_LIB = os.path.join(HERE, "libsmcsd_testing.so")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

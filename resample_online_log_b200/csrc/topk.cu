@@ -525,19 +525,6 @@ extern "C" sd_status gumbel_topk(const void* z, sd_dtype dt, int rows, int V, in
 
 // Draft step: one token per row from q_D = softmax(zD / tau) by Gumbel-max, which
 // is Gumbel-top-1: the dense kernel with k = 1 on its own noise stream.
-extern "C" sd_status sd_draft_sample(const void* zD, sd_dtype dt, int rows, int V, int64_t ld,
-                                     float tau, uint64_t seed, uint64_t round, uint32_t row0,
-                                     int32_t* tokens_out, float* logq_out, uint32_t* dev_err,
-                                     void* stream) {
-  if (rows < 0 || V < 1 || ld < V || !(tau > 0.f && tau < INFINITY)) return SD_ERR_INVALID_ARG;
-  if (dt != SD_F32 && dt != SD_BF16) return SD_ERR_INVALID_ARG;
-  if (rows == 0) return SD_OK;
-  if (!zD || !tokens_out) return SD_ERR_INVALID_ARG;
-  if ((uint64_t)row0 + (uint64_t)rows > 0x100000000ull) return SD_ERR_INVALID_ARG;
-  return launch_topk_dense(zD, dt, rows, V, ld, 1, tau, seed, round, SD_STREAM_DRAFT, row0,
-                           tokens_out, nullptr, logq_out, dev_err, (cudaStream_t)stream);
-}
-
 extern "C" sd_status gumbel_topk_sparse(const int32_t* idx, const float* prob, int rows, int L,
                                         int k, float tau, uint64_t seed, uint64_t round,
                                         int32_t* idx_out, uint32_t* dev_err, void* stream) {

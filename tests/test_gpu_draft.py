@@ -1,5 +1,5 @@
-"""GPU parity of sd_draft_sample (the draft step's Gumbel-max sampler) against the
-oracle, through the C ABI."""
+"""GPU parity of sd_draft_sample (the draft step's two-level Gumbel-max sampler)
+against the oracle, through the C ABI."""
 
 import numpy as np
 import pytest
@@ -81,3 +81,39 @@ def test_draft_config_rows_sampled():
         assert np.array_equal(zr, zD[r].float().cpu().numpy()[None, :])
         o = oracle.sd_draft_sample(zr, cfg.tau, cfg.seed, 11, row0=int(r))
         discrete(tok[r:r + 1].cpu().numpy(), o["tokens"], o["margin"], f"draft_row{r}")
+
+
+@pytest.mark.parametrize("V", [1, 128, 129, 256, 300])
+def test_draft_block_boundaries(V):
+    rng = np.random.default_rng(V + 3)
+    z = (rng.standard_normal((40, V)) * 2).astype(np.float32)
+    tok, lq, err = run_draft(to_dev(z), 0.9, 1, 2)
+    o = oracle.sd_draft_sample(z, 0.9, 1, 2)
+    discrete(tok.cpu().numpy(), o["tokens"], o["margin"], f"draft{V}")
+    assert err == 0
+
+
+def test_draft_nan_behind_masked_entries():
+    z = np.zeros((2, 2000), dtype=np.float32)
+    z[0, 0] = np.nan
+    z[0, 1:8] = -np.inf
+    z[1, 520] = np.nan                     # second tile of a warp, first one masked
+    z[1, 512:520] = -np.inf
+    tok, lq, err = run_draft(to_dev(z), 1.0, 3, 3)
+    assert err == oracle.DEV_NONFINITE and tok.cpu().tolist() == [-1, -1]
+
+
+def test_draft_block_near_tie_settled_in_fp64():
+    """Two live blocks whose perturbed log-masses coincide to fp32 precision:
+    the fp32 bounds cannot settle the block, the fp64 path must, as the oracle."""
+    from oracle.philox import STREAM_DRAFT_BLOCK, gumbel_from_uniform, stream_words, uniform_from_bits
+    rows, V = 16, 256
+    z = np.zeros((rows, V), dtype=np.float32)
+    for r in range(rows):
+        gam = gumbel_from_uniform(uniform_from_bits(stream_words(5, 8, STREAM_DRAFT_BLOCK, r, 2)))
+        z[r, :128] = 1.0
+        z[r, 128:] = np.float32(1.0 + (gam[0] - gam[1]))   # lambda_1 + G_1 ~= lambda_0 + G_0
+    tok, lq, err = run_draft(to_dev(z), 1.0, 5, 8)
+    o = oracle.sd_draft_sample(z, 1.0, 5, 8)
+    discrete(tok.cpu().numpy(), o["tokens"], o["margin"], "near-tie")
+    assert err == 0 and bool((tok >= 0).all())

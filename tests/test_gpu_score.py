@@ -263,3 +263,21 @@ def test_log_potential(with_prev):
         assert np.array_equal(g[k], g0[k]), k
     fin = np.isfinite(phi)
     assert np.allclose((g["logw"] - g0["logw"])[fin], phi[fin], atol=1e-12, rtol=0)
+
+
+def test_bonus_block_near_tie_settled_in_fp64():
+    """The bonus row's two live blocks tie to fp32 precision after their block
+    noise: the leader must settle the block in fp64, as the oracle does."""
+    from oracle.philox import STREAM_BONUS_BLOCK, gumbel_from_uniform, stream_words, uniform_from_bits
+    B, N, K, V = 1, 8, 1, 256
+    rng = np.random.default_rng(77)
+    zT = rng.standard_normal((B, N, K + 1, V)).astype(np.float32)
+    for n in range(N):
+        gam = gumbel_from_uniform(uniform_from_bits(stream_words(6, 2, STREAM_BONUS_BLOCK, n, 2)))
+        zT[0, n, K, :128] = 0.5
+        zT[0, n, K, 128:] = np.float32(0.5 + (gam[0] - gam[1]))
+    zD = zT.copy()
+    x = rng.integers(0, V, size=(B, N, K)).astype(np.int32)
+    g = run_score(zT, zD, x, 1.0, 6, 2, dtype="f32")
+    o = oracle.smcsd_score(zT, zD, x, 1.0, 6, 2)
+    compare(g, o, "bonus-near-tie")

@@ -42,6 +42,7 @@ STREAM_TOPK_SPARSE = 6  # sparse Gumbel-top-k noise (per stored entry)
 STREAM_DRAFT = 8        # draft-token Gumbel noise of the draft step (per vocabulary entry)
 STREAM_BONUS_BLOCK = 9  # bonus-token Gumbel noise per block of 128 entries (two-level draw)
 STREAM_DRAFT_BLOCK = 10  # draft-token Gumbel noise per block of 128 entries (two-level draw)
+STREAM_TOPK_BLOCK = 11  # dense Gumbel-top-k: block-maximum noise per block of 128 entries
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1):

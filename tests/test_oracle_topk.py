@@ -84,3 +84,48 @@ def test_sparse_first_pick_law():
     counts = np.bincount(out["idx"][:, 0] - 1000, minlength=L)
     _, pval = stats.chisquare(counts, prob * M)
     assert pval > 1e-3
+
+
+def test_plackett_luce_pairs_across_blocks_v600_k2():
+    """Five blocks of the top-down draw: ordered first-two picks over six heavy
+    tokens in different blocks and the pooled rest follow Plackett-Luce."""
+    V, M = 600, 30000
+    z = np.full(V, -1.0)
+    heavy = [5, 140, 260, 262, 390, 599]          # blocks 0, 1, 2, 2, 3, 4
+    z[heavy] = [2.5, 2.0, 1.8, 1.5, 2.2, 1.0]
+    tau = 1.0
+    s = z / np.float64(np.float32(tau))
+    p = _softmax(s)
+    out = oracle.gumbel_topk(np.broadcast_to(z, (M, V)), 2, tau, seed=8, rnd=3)
+    cat = np.full(V, len(heavy))
+    cat[heavy] = np.arange(len(heavy))
+    C = len(heavy) + 1
+    pairs = cat[out["idx"][:, 0]] * C + cat[out["idx"][:, 1]]
+    counts = np.bincount(pairs, minlength=C * C).astype(float)
+    expect = np.zeros(C * C)
+    for u in range(V):
+        for w in range(V):
+            if u != w:
+                expect[cat[u] * C + cat[w]] += p[u] * p[w] / (1 - p[u])
+    expect *= M
+    mask = expect > 5
+    assert counts[~mask].sum() <= 5 * (~mask).sum() + 20
+    _, pval = stats.chisquare(counts[mask], expect[mask] * counts[mask].sum() / expect[mask].sum())
+    assert pval > 1e-3, pval
+
+
+def test_conditioned_scores_keep_order_and_hit_the_block_maximum():
+    from oracle.topk import _conditioned_scores
+    rng = np.random.default_rng(4)
+    h = rng.gumbel(size=128) + rng.standard_normal(128)
+    h[[3, 50]] = -np.inf
+    S = _conditioned_scores(h, 7.25)
+    z = int(np.argmax(h))
+    assert S[z] == 7.25 and np.all(S[np.arange(128) != z] < 7.25)
+    live = np.isfinite(h)
+    assert np.array_equal(np.argsort(-h[live], kind="stable"), np.argsort(-S[live], kind="stable"))
+    assert np.all(S[[3, 50]] == -np.inf)
+    # -log(e^{-M} - e^{-Z} + e^{-h}) written directly, where it is well conditioned
+    Zm = h.max()
+    direct = -np.log(np.exp(-7.25) - np.exp(-Zm) + np.exp(-h[live]))
+    assert np.allclose(S[live], direct, rtol=1e-10, atol=1e-10)

@@ -91,6 +91,7 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_STREAM_DRAFT 8u
 #define SD_STREAM_BONUS_BLOCK 9u
 #define SD_STREAM_DRAFT_BLOCK 10u
+#define SD_STREAM_TOPK_BLOCK 11u
 
 /*
  * smcsd_score -- scoring step of one SMC-SD round ([SMC-SD] section 2, scoring
@@ -232,13 +233,21 @@ SMCSD_API sd_status sd_verify_reject(const void* zT, const void* zD, sd_dtype dt
 
 /*
  * gumbel_topk -- k tokens per row without replacement by Gumbel-top-k
- * ([STAND] Methodology item 2): the k largest s_v + g_v, s = z/tau, g from
- * stream 5 with row id = row, descending, ties to the lower v.
+ * ([STAND] Methodology item 2), drawn top-down over blocks of 128 entries
+ * (s = z/tau, row id = row):
+ *   M_j = log sum_{v in j} e^{s_v} + G_j, G from stream 11 (counter entry j);
+ *   the k largest M_j are kept (ties to the lower j);
+ *   in a kept block, h_v = s_v + g_v (g from stream 5, counter entry v),
+ *   Z_j = max h, and S_v = -log(e^{-M_j} - e^{-Z_j} + e^{-h_v}) (Gumbels
+ *   conditioned on the block's maximum M_j);
+ *   output the k largest S_v, descending, ties to the lower v.
+ * The law is that of one independent Gumbel per entry (k draws without
+ * replacement from softmax(s)); with V <= 128 the order is that of s_v + g_v.
  * z          device [rows, V] at row stride ld, dtype dt.
  * idx_out    device int32 [rows, k] (required).
- * score_out  device fp32 [rows, k]: s_v + g_v (or NULL).
+ * score_out  device fp32 [rows, k]: S_v (or NULL).
  * logp_out   device fp32 [rows, k]: s_v - logsumexp(s) (or NULL).
- * Requirements: rows >= 0, 1 <= k <= 16, k <= V, ld >= V.
+ * Requirements: rows >= 0, 1 <= k <= 16, k <= V <= 262144, ld >= V.
  * Faults: rows with NaN / +inf or all -inf -> SD_DEV_NONFINITE, ids -1;
  *   ranks with no finite entry left are -1.
  */

@@ -64,12 +64,14 @@ def test_dense_peaked_and_masked_rows():
     assert list(g["idx"][1, 3:]) == [-1] * 5
 
 
-def check_all_rows(z, cfg, idx, sc, lp):
+def check_all_rows(z, cfg, idx, sc, lp, seed, rnd):
     """Identities every row of the whole config must satisfy (the oracle covers
     sampled rows): indices in range and distinct; logp = z[idx]/tau - lse (a
-    gather of the input and the row's log-sum-exp, fp64); score - z[idx]/tau is a
-    Gumbel of a 23-bit uniform, so it lies in [g_min, g_max]; scores are
-    non-increasing along k."""
+    gather of the input and the row's log-sum-exp, fp64); each score is at most
+    its block's maximum M_j = log sum_{v in j} e^{z_v/tau} + G_j (block noise
+    from the oracle's generator) and the first equals its block's maximum;
+    scores are non-increasing along k."""
+    from oracle.philox import STREAM_TOPK_BLOCK, gumbel_from_uniform, stream_words, uniform_from_bits
     rows, V = z.shape
     tau = float(np.float32(cfg.tau))  # the C ABI takes tau in fp32
     assert bool(((idx >= 0) & (idx < V)).all()), "topk: index out of range"
@@ -80,9 +82,20 @@ def check_all_rows(z, cfg, idx, sc, lp):
     a = z.gather(1, idx.long()).double() / tau
     dl = (lp.double() - (a - lse[:, None])).abs()
     assert bool((dl <= 1e-5 * (1.0 + a.abs())).all()), f"topk: logp off by {float(dl.max()):.3e}"
-    g = sc.double() - a
-    g_min, g_max = -2.8104282144774236, 16.635532333438686
-    assert bool(((g >= g_min - 1e-4) & (g <= g_max + 1e-4)).all()), "topk: score - z/tau not a Gumbel"
+    nb = (V + 127) // 128
+    lam = []
+    for r0 in range(0, rows, 256):
+        zz = torch.full((min(256, rows - r0), nb * 128), -float("inf"), dtype=torch.float64, device=z.device)
+        zz[:, :V] = z[r0:r0 + 256].double() / tau
+        lam.append(torch.logsumexp(zz.view(-1, nb, 128), dim=2))
+    lam = torch.cat(lam)
+    G = torch.from_numpy(gumbel_from_uniform(uniform_from_bits(
+        stream_words(seed, rnd, STREAM_TOPK_BLOCK, np.arange(rows), nb)))).to(z.device)
+    Mj = (lam + G).gather(1, (idx.long() // 128))
+    s64 = sc.double()
+    assert bool((s64 <= Mj + 1e-4 * (1 + Mj.abs())).all()), "topk: a score above its block's maximum"
+    assert bool(((s64[:, 0] - Mj[:, 0]).abs() <= 1e-4 * (1 + Mj[:, 0].abs())).all()), \
+        "topk: the first score is not its block's maximum"
     assert bool((sc[:, 1:] <= sc[:, :-1]).all()), "topk: scores not in descending order"
 
 
@@ -101,7 +114,7 @@ def test_dense_config_sampled():
     lib.gumbel_topk(z, cfg.topk, cfg.tau, cfg.seed, 2, idx, score_out=sc, logp_out=lp, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    check_all_rows(z, cfg, idx, sc, lp)
+    check_all_rows(z, cfg, idx, sc, lp, cfg.seed, 2)
     for r in [0, 1, 2047, 4095]:
         h = gen.gen_config_rows(cfg, seqs=[r])
         assert np.array_equal(z[r].float().cpu().numpy(), h["z"][0])

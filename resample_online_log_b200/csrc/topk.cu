@@ -92,6 +92,162 @@ __device__ double block_max64(const TIn* row, int V, int j, double tau64, const 
   return m + log(sum) + gumbel_f64(uniform_f64(word_of(w, j & 3)));
 }
 
+// The k largest block maxima of the row (kept blocks and their fp64 maxima
+// into sm.keep / sm.keepM / sm.nkeep).  Every thread of the CTA calls it.
+template <typename TIn>
+__device__ __noinline__ void topk_keep_blocks(TopkSmem& sm, const TIn* row, int V, int nb, int k,
+                                              double tau64, const Stream& sblk, uint32_t rid,
+                                              bool rowbad) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // ---------------- blocks: the k largest maxima
+  float lo_t = -INFINITY;  // this thread's best lower bound
+  for (int j = tid; j < nb; j += kTThreads) lo_t = fmaxf(lo_t, sm.bs[j] - sm.bd[j]);
+  const float T = cta_kth_largest(lo_t, k, sm.kbuf);  // (syncs the CTA)
+  if (!rowbad) {
+    for (int j = tid; j < nb; j += kTThreads) {
+      if (sm.bs[j] > -INFINITY && sm.bs[j] + sm.bd[j] >= T) {
+        const int pos = atomicAdd(&sm.ncand, 1);
+        if (pos < kTCand) sm.cblk[pos] = j;
+        else atomicOr(&sm.flag, 2);
+      }
+    }
+  }
+  __syncthreads();
+  const int nc = min(sm.ncand, kTCand);
+  const bool overflow = (sm.flag & 2) != 0;
+  // fp32 ranks of the candidates (score, then lower block); bounds decide
+  if (!rowbad && !overflow && tid < nc) {
+    const int j = sm.cblk[tid];
+    const float sj = sm.bs[j];
+    int rk = 0;
+    for (int c = 0; c < nc; ++c) {
+      const int o = sm.cblk[c];
+      const float so = sm.bs[o];
+      rk += (so > sj || (so == sj && o < j)) ? 1 : 0;
+    }
+    sm.crank[tid] = rk;
+    if (rk < k) atomicMin(&sm.lo_ord, f2ord(sj - sm.bd[j]));
+    else atomicMax(&sm.hi_ord, f2ord(sj + sm.bd[j]));
+  }
+  __syncthreads();
+  if (!rowbad) {
+    const bool settled = !overflow && ord2f(sm.lo_ord) > ord2f(sm.hi_ord);
+    if (settled) {
+      // the kept blocks: the k best; their fp64 maxima, a warp each
+      if (tid < nc && sm.crank[tid] < k) sm.keep[sm.crank[tid]] = sm.cblk[tid];
+      if (tid == 0) sm.nkeep = min(nc, k);
+      __syncthreads();
+      for (int q = warp; q < sm.nkeep; q += kTWarps) {
+        const double m64 = block_max64<TIn>(row, V, sm.keep[q], tau64, sblk, rid);
+        if (lane == 0) sm.keepM[q] = m64;
+      }
+    } else if (!overflow) {
+      // fp64 maxima of the candidates, ranked exactly (score, then lower block)
+      for (int c = warp; c < nc; c += kTWarps) {
+        const double m64 = block_max64<TIn>(row, V, sm.cblk[c], tau64, sblk, rid);
+        if (lane == 0) sm.cM[c] = m64;
+      }
+      __syncthreads();
+      if (tid < nc) {
+        const int j = sm.cblk[tid];
+        const double sj = sm.cM[tid];
+        int rk = 0;
+        for (int c = 0; c < nc; ++c) {
+          const int o = sm.cblk[c];
+          const double so = sm.cM[c];
+          rk += (so > sj || (so == sj && o < j)) ? 1 : 0;
+        }
+        if (rk < k && sj > -INFINITY) {
+          sm.keep[rk] = j;
+          sm.keepM[rk] = sj;
+        }
+      }
+      if (tid == 0) {
+        int n = 0;
+        for (int c = 0; c < nc; ++c) n += sm.cM[c] > -INFINITY ? 1 : 0;
+        sm.nkeep = min(n, k);
+      }
+    } else {
+      // more candidates than the table holds (ties flooding the bound):
+      // fp64 maxima of every block (in the entry table), k rounds of arg-max
+      for (int j = warp; j < nb; j += kTWarps) {
+        const double m64 = block_max64<TIn>(row, V, j, tau64, sblk, rid);
+        if (lane == 0) sm.es[j] = m64;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int taken = 0;
+        for (int q = 0; q < k; ++q) {
+          double best = -INFINITY;
+          int bi = 0x7FFFFFFF;
+          for (int j = lane; j < nb; j += 32) {
+            bool used = false;
+            for (int p = 0; p < taken; ++p) used |= sm.keep[p] == j;
+            if (!used) c64_merge(best, bi, sm.es[j], j);
+          }
+          warp_c64(best, bi);
+          if (bi == 0x7FFFFFFF || !(best > -INFINITY)) break;
+          if (lane == 0) {
+            sm.keep[taken] = bi;
+            sm.keepM[taken] = best;
+          }
+          __syncwarp();
+          ++taken;
+        }
+        if (lane == 0) sm.nkeep = taken;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Entry scores of the kept blocks conditioned on their maxima, fp64, a warp
+// per block; those at or above the smallest kept maximum go to sm.es / sm.ei.
+template <typename TIn>
+__device__ __noinline__ void topk_kept_entries(TopkSmem& sm, const TIn* row, int V, int k,
+                                               double tau64, const Stream& sent, uint32_t rid,
+                                               bool rowbad) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // ---------------- entries of the kept blocks (fp64), a warp per block
+  const int nk = rowbad ? 0 : sm.nkeep;
+  double Tm = INFINITY;  // the k-th largest score is no smaller than the smallest kept maximum
+  for (int q = 0; q < nk; ++q) Tm = fmin(Tm, sm.keepM[q]);
+  if (nk < k) Tm = -INFINITY;  // fewer live blocks than k: every entry counts
+  for (int q = warp; q < nk; q += kTWarps) {
+    const int j = sm.keep[q];
+    const double Mj = sm.keepM[q];
+    const int v0 = j * kTBlk + 4 * lane;
+    double h[4];
+    U4 w = U4{0u, 0u, 0u, 0u};
+    if (v0 < V) w = sent.at((uint32_t)(v0 >> 2), rid);
+    double Z = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float zv = v0 + t < V ? ld_elem<TIn>(row, v0 + t) : -INFINITY;
+      h[t] = zv > -INFINITY ? (double)zv / tau64 + gumbel_f64(uniform_f64(word_of(w, t))) : -INFINITY;
+      Z = fmax(Z, h[t]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Z = fmax(Z, __shfl_xor_sync(0xffffffffu, Z, o));
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      if (!(h[t] > -INFINITY)) continue;
+      // S = -log(e^{-M} - e^{-Z} + e^{-h}) = M - softplus(M - h + log(1 - e^{h - Z}))
+      double sv = Mj;
+      const double d = h[t] - Z;
+      if (d != 0.0) {
+        const double u = Mj - h[t] + log(-expm1(d));
+        sv = Mj - (fmax(u, 0.0) + log1p(exp(-fabs(u))));
+      }
+      if (sv >= Tm) {
+        const int pos = atomicAdd(&sm.ne, 1);
+        sm.es[pos] = sv;
+        sm.ei[pos] = v0 + t;
+      }
+    }
+  }
+}
+
 template <typename TIn>
 __global__ void __launch_bounds__(kTThreads, 2) topk_block_kernel(
     const TIn* __restrict__ z, int rows, int V, int64_t ld, int k, float inv_tau, float cT,
@@ -215,145 +371,11 @@ __global__ void __launch_bounds__(kTThreads, 2) topk_block_kernel(
         if (!(MM > -INFINITY)) sm.flag |= 1;  // every entry -inf
       }
     }
-    // ---------------- blocks: the k largest maxima
-    float lo_t = -INFINITY;  // this thread's best lower bound
-    for (int j = tid; j < nb; j += kTThreads) lo_t = fmaxf(lo_t, sm.bs[j] - sm.bd[j]);
-    const float T = cta_kth_largest(lo_t, k, sm.kbuf);  // (syncs the CTA)
+    __syncthreads();
     const bool rowbad = (sm.flag & 1) != 0;
-    if (!rowbad) {
-      for (int j = tid; j < nb; j += kTThreads) {
-        if (sm.bs[j] > -INFINITY && sm.bs[j] + sm.bd[j] >= T) {
-          const int pos = atomicAdd(&sm.ncand, 1);
-          if (pos < kTCand) sm.cblk[pos] = j;
-          else atomicOr(&sm.flag, 2);
-        }
-      }
-    }
+    topk_keep_blocks<TIn>(sm, row, V, nb, k, tau64, sblk, rid, rowbad);
     __syncthreads();
-    const int nc = min(sm.ncand, kTCand);
-    const bool overflow = (sm.flag & 2) != 0;
-    // fp32 ranks of the candidates (score, then lower block); bounds decide
-    if (!rowbad && !overflow && tid < nc) {
-      const int j = sm.cblk[tid];
-      const float sj = sm.bs[j];
-      int rk = 0;
-      for (int c = 0; c < nc; ++c) {
-        const int o = sm.cblk[c];
-        const float so = sm.bs[o];
-        rk += (so > sj || (so == sj && o < j)) ? 1 : 0;
-      }
-      sm.crank[tid] = rk;
-      if (rk < k) atomicMin(&sm.lo_ord, f2ord(sj - sm.bd[j]));
-      else atomicMax(&sm.hi_ord, f2ord(sj + sm.bd[j]));
-    }
-    __syncthreads();
-    if (!rowbad) {
-      const bool settled = !overflow && ord2f(sm.lo_ord) > ord2f(sm.hi_ord);
-      if (settled) {
-        // the kept blocks: the k best; their fp64 maxima, a warp each
-        if (tid < nc && sm.crank[tid] < k) sm.keep[sm.crank[tid]] = sm.cblk[tid];
-        if (tid == 0) sm.nkeep = min(nc, k);
-        __syncthreads();
-        for (int q = warp; q < sm.nkeep; q += kTWarps) {
-          const double m64 = block_max64<TIn>(row, V, sm.keep[q], tau64, sblk, rid);
-          if (lane == 0) sm.keepM[q] = m64;
-        }
-      } else if (!overflow) {
-        // fp64 maxima of the candidates, ranked exactly (score, then lower block)
-        for (int c = warp; c < nc; c += kTWarps) {
-          const double m64 = block_max64<TIn>(row, V, sm.cblk[c], tau64, sblk, rid);
-          if (lane == 0) sm.cM[c] = m64;
-        }
-        __syncthreads();
-        if (tid < nc) {
-          const int j = sm.cblk[tid];
-          const double sj = sm.cM[tid];
-          int rk = 0;
-          for (int c = 0; c < nc; ++c) {
-            const int o = sm.cblk[c];
-            const double so = sm.cM[c];
-            rk += (so > sj || (so == sj && o < j)) ? 1 : 0;
-          }
-          if (rk < k && sj > -INFINITY) {
-            sm.keep[rk] = j;
-            sm.keepM[rk] = sj;
-          }
-        }
-        if (tid == 0) {
-          int n = 0;
-          for (int c = 0; c < nc; ++c) n += sm.cM[c] > -INFINITY ? 1 : 0;
-          sm.nkeep = min(n, k);
-        }
-      } else {
-        // more candidates than the table holds (ties flooding the bound):
-        // fp64 maxima of every block (in the entry table), k rounds of arg-max
-        for (int j = warp; j < nb; j += kTWarps) {
-          const double m64 = block_max64<TIn>(row, V, j, tau64, sblk, rid);
-          if (lane == 0) sm.es[j] = m64;
-        }
-        __syncthreads();
-        if (warp == 0) {
-          int taken = 0;
-          for (int q = 0; q < k; ++q) {
-            double best = -INFINITY;
-            int bi = 0x7FFFFFFF;
-            for (int j = lane; j < nb; j += 32) {
-              bool used = false;
-              for (int p = 0; p < taken; ++p) used |= sm.keep[p] == j;
-              if (!used) c64_merge(best, bi, sm.es[j], j);
-            }
-            warp_c64(best, bi);
-            if (bi == 0x7FFFFFFF || !(best > -INFINITY)) break;
-            if (lane == 0) {
-              sm.keep[taken] = bi;
-              sm.keepM[taken] = best;
-            }
-            __syncwarp();
-            ++taken;
-          }
-          if (lane == 0) sm.nkeep = taken;
-        }
-      }
-    }
-    __syncthreads();
-    // ---------------- entries of the kept blocks (fp64), a warp per block
-    const int nk = rowbad ? 0 : sm.nkeep;
-    double Tm = INFINITY;  // the k-th largest score is no smaller than the smallest kept maximum
-    for (int q = 0; q < nk; ++q) Tm = fmin(Tm, sm.keepM[q]);
-    if (nk < k) Tm = -INFINITY;  // fewer live blocks than k: every entry counts
-    for (int q = warp; q < nk; q += kTWarps) {
-      const int j = sm.keep[q];
-      const double Mj = sm.keepM[q];
-      const int v0 = j * kTBlk + 4 * lane;
-      double h[4];
-      U4 w = U4{0u, 0u, 0u, 0u};
-      if (v0 < V) w = sent.at((uint32_t)(v0 >> 2), rid);
-      double Z = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float zv = v0 + t < V ? ld_elem<TIn>(row, v0 + t) : -INFINITY;
-        h[t] = zv > -INFINITY ? (double)zv / tau64 + gumbel_f64(uniform_f64(word_of(w, t))) : -INFINITY;
-        Z = fmax(Z, h[t]);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) Z = fmax(Z, __shfl_xor_sync(0xffffffffu, Z, o));
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        if (!(h[t] > -INFINITY)) continue;
-        // S = -log(e^{-M} - e^{-Z} + e^{-h}) = M - softplus(M - h + log(1 - e^{h - Z}))
-        double sv = Mj;
-        const double d = h[t] - Z;
-        if (d != 0.0) {
-          const double u = Mj - h[t] + log(-expm1(d));
-          sv = Mj - (fmax(u, 0.0) + log1p(exp(-fabs(u))));
-        }
-        if (sv >= Tm) {
-          const int pos = atomicAdd(&sm.ne, 1);
-          sm.es[pos] = sv;
-          sm.ei[pos] = v0 + t;
-        }
-      }
-    }
+    topk_kept_entries<TIn>(sm, row, V, k, tau64, sent, rid, rowbad);
     __syncthreads();
     const int ne = rowbad ? 0 : sm.ne;
     for (int e = tid; e < ne; e += kTThreads) {  // ranks by counting (score, then lower index)

@@ -43,6 +43,7 @@ STREAM_DRAFT = 8        # draft-token Gumbel noise of the draft step (per vocabu
 STREAM_BONUS_BLOCK = 9  # bonus-token Gumbel noise per block of 128 entries (two-level draw)
 STREAM_DRAFT_BLOCK = 10  # draft-token Gumbel noise per block of 128 entries (two-level draw)
 STREAM_TOPK_BLOCK = 11  # dense Gumbel-top-k: block-maximum noise per block of 128 entries
+STREAM_RESIDUAL_BLOCK = 12  # verify residual draw: noise per block of 128 entries (two-level)
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1):

@@ -11,13 +11,16 @@ not print the rule; this is the textbook speculative-sampling rule:
       u_k ~ U(0,1) from Philox stream 2, row id b*(K+1)+k, c0 = 0, word 0
       accept iff u_k * q(x) < p(x)          (u < min(1, p/q) without a division)
   at the first reject j:
-      r_v = max(p_v - q_v, 0); emitted token = argmax_{v : r_v > 0} (log r_v + g_v)
-      with g_v from Philox stream 3, row id b*(K+1)+j (Gumbel-max over the
-      normalised residual; the normaliser does not change the argmax).
+      r_v = max(p_v - q_v, 0); the emitted token is a sample of the normalised
+      residual by the exact two-level Gumbel-max of ``oracle.blockdraw`` over
+      log r (block noise from Philox stream 12, entry noise from stream 3, row
+      id b*(K+1)+j): the 128-entry block by log sum r + G_j, then
+      argmax_{v : r_v > 0} (log r_v + g_v) inside it.
       If every r_v = 0 the zero-residual error bit is raised and the token is
-      drawn from p with the same noise.
-  if all K are accepted: bonus = argmax_v (z_T[K, v]/tau + g_v), Philox
-      stream 1, row id b.
+      drawn from p by the same draw over a = z/tau with the same streams.
+  if all K are accepted: the bonus token is the two-level draw over
+      a = z_T[K]/tau with block noise from stream 9 and entry noise from
+      stream 1, row id b (the SMC-SD bonus sampler).
   accepted_len = j (or K); out_tokens = accepted drafts + the one drawn token,
   padded with -1 to K+1 entries; tv[b, k] = 1/2 sum_v |p_v - q_v| at all k < K
   (METASD section 2, Block Divergence built on total variation).
@@ -36,10 +39,10 @@ enumeration at V = 4, K = 2 (the emitted token law equals the target law to
 
 import numpy as np
 
-from .philox import (STREAM_ACCEPT, STREAM_BONUS, STREAM_RESIDUAL, gumbel_from_uniform,
-                     row_scalar_word, stream_words, uniform_from_bits)
-from .score import (DEV_NONFINITE, DEV_TOKEN_OOB, DEV_ZERO_RESIDUAL, gumbel_argmax,
-                    row_log_softmax, total_variation)
+from .blockdraw import block_gumbel_argmax
+from .philox import (STREAM_ACCEPT, STREAM_BONUS, STREAM_BONUS_BLOCK, STREAM_RESIDUAL,
+                     STREAM_RESIDUAL_BLOCK, row_scalar_word, uniform_from_bits)
+from .score import DEV_NONFINITE, DEV_TOKEN_OOB, DEV_ZERO_RESIDUAL, row_log_softmax, total_variation
 
 
 def accept_probability(p, q, x):
@@ -107,16 +110,15 @@ def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd, b0=0):
             if accept:
                 out[b, k] = x
                 continue
-            g = gumbel_from_uniform(uniform_from_bits(
-                stream_words(seed, rnd, STREAM_RESIDUAL, (b0 + b) * R + k, V)))
             r = np.maximum(p - q, 0.0)
             if (r > 0).any():
                 with np.errstate(divide="ignore"):
-                    score = np.where(r > 0, np.log(r), -np.inf) + g
+                    w = np.where(r > 0, np.log(np.where(r > 0, r, 1.0)), -np.inf)
             else:
                 err |= DEV_ZERO_RESIDUAL
-                score = a[k] + g
-            tok, mg = gumbel_argmax(score)
+                w = a[k]
+            tok, mg = block_gumbel_argmax(w, seed, rnd, STREAM_RESIDUAL_BLOCK, STREAM_RESIDUAL,
+                                          (b0 + b) * R + k)
             out[b, k] = tok
             tok_margin[b] = mg
             acc_len[b] = k
@@ -128,8 +130,7 @@ def sd_verify_reject(zT, zD, draft_tokens, tau, seed, rnd, b0=0):
         if np.isnan(lse_t[K]):
             err |= DEV_NONFINITE
             continue
-        g = gumbel_from_uniform(uniform_from_bits(stream_words(seed, rnd, STREAM_BONUS, b0 + b, V)))
-        tok, mg = gumbel_argmax(a[K] + g)
+        tok, mg = block_gumbel_argmax(a[K], seed, rnd, STREAM_BONUS_BLOCK, STREAM_BONUS, b0 + b)
         out[b, K] = tok
         tok_margin[b] = mg
     return dict(accepted_len=acc_len, out_tokens=out, tv=tv, accept_margin=acc_margin,

@@ -3,7 +3,7 @@
 import itertools
 
 import numpy as np
-from scipy import stats
+from scipy import special, stats
 
 import oracle
 from oracle import score as osc
@@ -114,3 +114,27 @@ def test_bad_token_is_rejected():
     with np.errstate(divide="ignore"):
         expect = int(np.argmax(np.where(r > 0, np.log(r), -np.inf) + g))
     assert out["out_tokens"][0, 0] == expect
+
+
+def test_first_token_law_across_blocks_v700():
+    """Drafts x ~ q, target p over V = 700 (six blocks of the two-level residual
+    draw): the first emitted token (the accepted draft, or the residual draw
+    after a rejection) follows p; chi-square over 14 bins of 6000 sequences."""
+    V, B = 700, 6000
+    v = np.arange(V)
+    zt = 1.5 * np.sin(v / 41.0) + 0.5 * np.cos(v / 3.0)
+    zd = 1.5 * np.cos(v / 29.0)
+    p = np.exp(zt - special.logsumexp(zt))
+    q = np.exp(zd - special.logsumexp(zd))
+    rng = np.random.default_rng(17)
+    x = rng.choice(V, size=(B, 1), p=q)
+    zT = np.broadcast_to(np.stack([zt, zt]), (B, 2, V))
+    zD = np.broadcast_to(zd[None, None, :], (B, 1, V))
+    out = oracle.sd_verify_reject(zT, zD, x, 1.0, seed=3, rnd=1)
+    first = out["out_tokens"][:, 0]
+    assert (first >= 0).all()
+    bins = v // 50
+    counts = np.bincount(bins[first], minlength=14)
+    expect = np.bincount(bins, weights=p, minlength=14) * B
+    _, pval = stats.chisquare(counts, expect)
+    assert pval > 1e-3, pval

@@ -92,6 +92,7 @@ typedef enum sd_dtype { SD_F32 = 0, SD_BF16 = 1 } sd_dtype;
 #define SD_STREAM_BONUS_BLOCK 9u
 #define SD_STREAM_DRAFT_BLOCK 10u
 #define SD_STREAM_TOPK_BLOCK 11u
+#define SD_STREAM_RESIDUAL_BLOCK 12u
 
 /*
  * smcsd_score -- scoring step of one SMC-SD round ([SMC-SD] section 2, scoring

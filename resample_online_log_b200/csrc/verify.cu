@@ -6,44 +6,49 @@
 // K are accepted a bonus token is drawn from the target row K+1.  Sources:
 // "Faster LLM Inference via Sequential Monte Carlo", section 1 (standard SD,
 // rejection, KV rollback); METASD section 1 (background) and section 2 (TV
-// block divergence reported per position).
+// block divergence reported per position).  Both draws are exact two-level
+// Gumbel-max draws over blocks of 128 entries (the block by its log-mass plus
+// block noise, then the entry inside it).
 //
 // Design (B200, sm_100a).  Every (sequence, position) row is independent until
-// the first rejection is known, so each is scored on its own, all at once:
-//   verify_rows_kernel: one CTA of 1024 threads per row (a thread-block cluster
-//     of C CTAs when V exceeds one CTA's slice, the CTAs exchanging partials
-//     through distributed shared memory); each thread holds 32 bf16 (16 fp32)
-//     entries of the target and draft rows in registers, loaded with 16-byte
-//     vector loads.  Per row: the log-sum-exp of both rows (fp64 combine), the
-//     accept test u q(x) < p(x) in fp64, TV = 1/2 sum |p - q| (exps recomputed
-//     from the registers), and -- only if the row rejects its draft token --
-//     the residual draw argmax_{r_v > 0} (log r_v + g_v), r = max(p - q, 0);
-//     the last row draws the bonus token argmax (z/tau + g).  The draws are
-//     exact: an fp32 screen with rigorous error bounds keeps only entries that
-//     can still win, near-ties are re-scored in fp64 over the whole row.  Each
-//     row's outcome is encoded in its own slot of out_tokens.
+// the first rejection is known, so all rows are scored at once:
+//   verify_rows_kernel: persistent CTAs of 512 threads (two per SM) take rows
+//     in turn, streaming each row twice in tiles of 256 entries (8 per lane,
+//     16-byte loads, several tiles in flight):
+//     pass 1 (HBM; the row stays in L2): the log-sum-exp of the target and
+//       draft rows, exps relative to each warp's running max (one redux per
+//       tile); the accept test u q(x) < p(x) in fp64;
+//     pass 2 (L2): p and q per entry, TV = 1/2 sum |p - q|, and the block
+//       masses the row's draw needs -- residual sum max(p - q, 0) after a
+//       rejection (with the error bound 7.7e-6 (p + q) per entry), target
+//       mass on the last row -- parked per lane and scored per block one per
+//       lane every 16 tiles; the CTA merges the block candidates (a near-tie,
+//       or no residual mass in fp32, goes to fp64 over the row's blocks), and
+//       one warp draws the entry inside the chosen block in fp64.
+//     Each row's outcome is encoded in its own slot of out_tokens.
 //   verify_finalize_kernel: per sequence, the first rejection decides the
 //     accepted length and the emitted tokens; slots past it become -1.
 // Work for rows past the first rejection is spent speculatively; nothing but
 // the outputs is written to global memory.
-#include <algorithm>
 #include <cuda_runtime.h>
 
+#include "rowload.cuh"
 #include "rows.cuh"
 
 namespace smcsd {
 
-constexpr int kVThreads = 1024;
+constexpr int kVThreads = 512;
+constexpr int kVPerSM = 2;
 constexpr int kVWarps = kVThreads / 32;
-constexpr int kVChunks = 4;  // 16-byte chunks of each row per thread
+constexpr int kVBlk = 128;
+constexpr int kVBuf = 16;  // tiles a warp buffers before scoring their blocks
 
 struct VerifyArgs {
   const void* zT;
   const void* zD;
   int64_t ld;
-  int V, K, R;
-  int slice;   // entries of a row per CTA
-  int vec;     // 16-byte loads allowed
+  int B, V, K, R;
+  int vec;  // 16-byte loads allowed
   float inv_tau, cT;
   double tau64;
   const int32_t* draft;
@@ -54,22 +59,18 @@ struct VerifyArgs {
   uint32_t* dev_err;
 };
 
-// What a CTA publishes to the other CTAs of its row's cluster.
-struct alignas(16) VExch {
-  float mT, sT, mD, sD;  // (max, sum of exps relative to it) over the CTA's slice
-  float zxT, zxD;        // raw logits of the draft token (its owner CTA only)
-  int own, pad0;
-  float tvp, pad1, pad2, pad3;  // TV partial
-  Cand cand;             // best candidate of the CTA's screen
-};
-
 struct VSmem {
-  float red[4][kVWarps];
-  Cand wc[kVWarps];
-  Cand64 w64[kVWarps];
-  VExch ex;
+  float part[kVWarps][kVBuf][32];  // per lane: its 8 entries' block mass (residual or target)
+  float pq[kVWarps][kVBuf][32];    // per lane: its 8 entries' p + q (residual error bounds)
+  int tile[kVWarps][kVBuf];
+  float rm[2][kVWarps], rs[2][kVWarps];  // lse partials (target, draft)
+  float tv[kVWarps];
+  Cand cand[kVWarps];
+  double s64[kVWarps];
+  int i64[kVWarps];
   double lse[2];
-  int flag;
+  int flag;   // bit 0: target bad, 1: draft bad, 2: accept, 3: draft token out of range
+  int block;  // chosen block, -1: settle in fp64, -2: none
 };
 
 // Encoding of a row's outcome in its out_tokens slot, decoded by the finalize
@@ -80,429 +81,363 @@ __device__ __forceinline__ int encode_reject(int tok, bool oob, bool zr) {
   return -2 - (tok | (oob ? (1 << 29) : 0) | (zr ? (1 << 30) : 0));
 }
 
+// fp64 log-weight of entry v for the row's draw: mode 1 the residual
+// log max(p - q, 0) (-inf where zero), else the target's z/tau.
 template <typename TIn>
-struct VT;
-template <>
-struct VT<uint16_t> {
-  static constexpr int EPC = 8;  // entries per 16-byte chunk
-  static __device__ __forceinline__ float get(const uint4& v, int j) {
-    const uint32_t w = (j >> 1) == 0 ? v.x : ((j >> 1) == 1 ? v.y : ((j >> 1) == 2 ? v.z : v.w));
-    return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
-  }
-  static __device__ __forceinline__ uint4 load(const uint16_t* g, int e0, int len, bool vec) {
-    if (vec && e0 + 8 <= len) return *reinterpret_cast<const uint4*>(g + e0);
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = e0 + 2 * j < len ? (uint32_t)g[e0 + 2 * j] : 0xFF80u;
-      const uint32_t hi = e0 + 2 * j + 1 < len ? (uint32_t)g[e0 + 2 * j + 1] : 0xFF80u;
-      w[j] = lo | (hi << 16);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-  }
-};
-template <>
-struct VT<float> {
-  static constexpr int EPC = 4;
-  static __device__ __forceinline__ float get(const uint4& v, int j) {
-    return __uint_as_float(j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w)));
-  }
-  static __device__ __forceinline__ uint4 load(const float* g, int e0, int len, bool vec) {
-    if (vec && e0 + 4 <= len) return *reinterpret_cast<const uint4*>(g + e0);
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) w[j] = e0 + j < len ? __float_as_uint(g[e0 + j]) : 0xFF800000u;
-    return make_uint4(w[0], w[1], w[2], w[3]);
-  }
-};
-
-// CTA-wide reductions of four values (max, NaN-propagating) / (sum) through shared memory.
-__device__ __forceinline__ float4 cta_max4_nan(float4 v, VSmem* sm) {
-  float a[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) asm volatile("redux.sync.max.NaN.f32 %0, %0, 0xffffffff;" : "+f"(a[i]));
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0)
-    for (int i = 0; i < 4; ++i) sm->red[i][warp] = a[i];
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    a[i] = sm->red[i][lane];
-    asm volatile("redux.sync.max.NaN.f32 %0, %0, 0xffffffff;" : "+f"(a[i]));
-  }
-  return make_float4(a[0], a[1], a[2], a[3]);
-}
-__device__ __forceinline__ float4 cta_sum4(float4 v, VSmem* sm) {
-  float a[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = warp_sum(a[i]);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0)
-    for (int i = 0; i < 4; ++i) sm->red[i][warp] = a[i];
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = warp_sum(sm->red[i][lane]);
-  return make_float4(a[0], a[1], a[2], a[3]);
-}
-__device__ __forceinline__ Cand cta_cand(Cand c, VSmem* sm) {
-  c = warp_cand(c);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) sm->wc[warp] = c;
-  __syncthreads();
-  return warp_cand(sm->wc[lane]);
+__device__ __forceinline__ double draw_weight64(const TIn* rT, const TIn* rD, int v, int mode,
+                                                double tau64, double lseT, double lseD) {
+  const double a = (double)ld_elem<TIn>(rT, v) / tau64;
+  if (mode != 1) return a;
+  const double r = exp(a - lseT) - exp((double)ld_elem<TIn>(rD, v) / tau64 - lseD);
+  return r > 0.0 ? log(r) : -INFINITY;
 }
 
-// Exact fp64 draw over a whole row, by the whole CTA (a near-tie the fp32
-// screens could not settle, or a zero residual; rare).  mode 0: argmax z/tau +
-// g; mode 1: argmax over max(p - q, 0) > 0 of log(p - q) + g.  Entries whose
-// fp32 upper bound stays below lo_star cannot win and are not re-scored.
+// The block of the draw in fp64 over the whole row (a near-tie the fp32 bounds
+// could not settle, or no residual mass in fp32; rare): every thread takes
+// whole blocks.  Returns the block, or -1 if no block has positive mass.
 template <typename TIn>
-__device__ __noinline__ int exact_draw_row(const TIn* rT, const TIn* rD, int V, int mode,
-                                           double lseT, double lseD, const VerifyArgs& a,
-                                           float lo_star, const Stream st, uint32_t rowid,
-                                           VSmem* sm) {
+__device__ __noinline__ int exact_block(VSmem& sm, const TIn* rT, const TIn* rD, int V, int mode,
+                                        double tau64, double lseT, double lseD, const Stream& sb,
+                                        uint32_t rid) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nb = (V + kVBlk - 1) / kVBlk;
   double best = -INFINITY;
   int bi = 0x7FFFFFFF;
-  for (int q = threadIdx.x; q * 4 < V; q += blockDim.x) {
-    const U4 w = st.at((uint32_t)q, rowid);
-    for (int j = 0; j < 4; ++j) {
-      const int v = q * 4 + j;
-      if (v >= V) break;
-      const float zt = Elem<TIn>::get(rT, v);
-      const float u = uniform_f32(word_of(w, j));
-      float hi;
-      if (mode == 0) {
-        const float a32 = zt * a.inv_tau;
-        if (!(a32 + kGumbelMaxF + 1e-3f >= lo_star)) continue;
-        const float g32 = gumbel_f32(u);
-        hi = a32 + g32 + score_err(a32, g32);
-      } else {
-        const float p = (float)exp((double)zt / a.tau64 - lseT);
-        const float q = (float)exp((double)Elem<TIn>::get(rD, v) / a.tau64 - lseD);
-        const float r = p - q, eb = 7.7e-6f * (p + q) + 1e-37f;
-        if (!(r + eb > 0.f)) continue;
-        const float lh = logf(r + eb);
-        if (!(lh + kGumbelMaxF + 1e-3f >= lo_star)) continue;
-        const float g32 = gumbel_f32(u);
-        hi = lh + g32 + score_err(lh, g32);
-      }
-      if (!(hi >= lo_star)) continue;
-      const double g64 = gumbel_f64(uniform_f64(word_of(w, j)));
-      double sv;
-      if (mode == 0) {
-        sv = (double)zt / a.tau64 + g64;
-      } else {
-        const double rr = exp((double)zt / a.tau64 - lseT) - exp((double)Elem<TIn>::get(rD, v) / a.tau64 - lseD);
-        sv = rr > 0.0 ? log(rr) + g64 : -INFINITY;
-      }
-      c64_merge(best, bi, sv, v);
+  for (int j = tid; j < nb; j += kVThreads) {
+    const int v0 = j * kVBlk, v1 = min(v0 + kVBlk, V);
+    double m = -INFINITY;
+    for (int v = v0; v < v1; ++v) m = fmax(m, draw_weight64<TIn>(rT, rD, v, mode, tau64, lseT, lseD));
+    if (!(m > -INFINITY)) continue;
+    double sum = 0.0;
+    for (int v = v0; v < v1; ++v) sum += exp(draw_weight64<TIn>(rT, rD, v, mode, tau64, lseT, lseD) - m);
+    const U4 w = sb.at((uint32_t)(j >> 2), rid);
+    c64_merge(best, bi, m + log(sum) + gumbel_f64(uniform_f64(word_of(w, j & 3))), j);
+  }
+  warp_c64(best, bi);
+  if (lane == 0) {
+    sm.s64[warp] = best;
+    sm.i64[warp] = bi;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    best = lane < kVWarps ? sm.s64[lane] : -INFINITY;
+    bi = lane < kVWarps ? sm.i64[lane] : 0x7FFFFFFF;
+    warp_c64(best, bi);
+    if (lane == 0) sm.block = bi == 0x7FFFFFFF ? -1 : bi;
+  }
+  __syncthreads();
+  return sm.block;
+}
+
+// The entry inside block j, in fp64 (one warp, four entries a lane).
+template <typename TIn>
+__device__ __noinline__ int exact_in_block(const TIn* rT, const TIn* rD, int V, int j, int mode,
+                                           double tau64, double lseT, double lseD,
+                                           const Stream& se, uint32_t rid) {
+  const int lane = threadIdx.x & 31;
+  const int v0 = j * kVBlk + 4 * lane;
+  double best = -INFINITY;
+  int bi = 0x7FFFFFFF;
+  if (v0 < V) {
+    const U4 w = se.at((uint32_t)(v0 >> 2), rid);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      if (v0 + t >= V) break;
+      const double wv = draw_weight64<TIn>(rT, rD, v0 + t, mode, tau64, lseT, lseD);
+      if (wv > -INFINITY) c64_merge(best, bi, wv + gumbel_f64(uniform_f64(word_of(w, t))), v0 + t);
     }
   }
   warp_c64(best, bi);
+  return bi == 0x7FFFFFFF ? -1 : bi;
+}
+
+// Pass 1 over a row pair (HBM; the rows are left in L2 for pass 2): per warp
+// the target's and draft's running max and sums of exps relative to it, and
+// NaN / +inf flags, into shared memory.
+template <typename TIn>
+__device__ __noinline__ void verify_pass1(VSmem& sm, const TIn* rT, const TIn* rD, int V, int nt,
+                                          bool hasD, float cT, bool vec, uint64_t keep) {
+  constexpr int kUnroll = sizeof(TIn) == 2 ? 2 : 1;  // tiles in flight per tensor (32 bytes a lane)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) {
-    sm->w64[warp].s = best;
-    sm->w64[warp].idx = bi;
+  // ---------------- pass 1 (HBM): the two rows' log-sum-exp
+  float RT = -INFINITY, RD = -INFINITY, ST = 0.f, SD = 0.f;
+  bool badT = false, badD = false;
+  for (int t0 = warp; t0 < nt; t0 += kUnroll * kVWarps) {
+    Raw8<TIn> xt[kUnroll], xd[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = t0 + u * kVWarps;
+      if (t < nt) {
+        xt[u] = load8_raw<TIn>(rT, t * 256 + 8 * lane, V, vec, keep);
+        if (hasD) xd[u] = load8_raw<TIn>(rD, t * 256 + 8 * lane, V, vec, keep);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (t0 + u * kVWarps >= nt) break;  // warp-uniform
+      float zt[8], zd[8];
+      unpack8<TIn>(xt[u], zt);
+      float mt = -INFINITY, md = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mt = fmax_nan(mt, zt[i]);
+      if (hasD) {
+        unpack8<TIn>(xd[u], zd);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) md = fmax_nan(md, zd[i]);
+      }
+      badT |= mt != mt;
+      badD |= md != md;
+      mt = mt != mt ? -INFINITY : mt;
+      md = md != md ? -INFINITY : md;
+      warp_max2(mt, md);
+      badT |= mt == INFINITY;
+      badD |= md == INFINITY;
+      if (mt > RT) {
+        ST = RT == -INFINITY ? 0.f : ST * ex2((RT - mt) * cT);
+        RT = mt;
+      }
+      if (RT > -INFINITY && RT < INFINITY) {
+        const float n = -RT * cT;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ST += ex2(fmaf(zt[i], cT, n));
+      }
+      if (hasD) {
+        if (md > RD) {
+          SD = RD == -INFINITY ? 0.f : SD * ex2((RD - md) * cT);
+          RD = md;
+        }
+        if (RD > -INFINITY && RD < INFINITY) {
+          const float n = -RD * cT;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) SD += ex2(fmaf(zd[i], cT, n));
+        }
+      }
+    }
   }
-  __syncthreads();
-  double s = lane < (int)(blockDim.x >> 5) ? sm->w64[lane].s : -INFINITY;
-  int i = lane < (int)(blockDim.x >> 5) ? sm->w64[lane].idx : 0x7FFFFFFF;
-  warp_c64(s, i);
-  return i == 0x7FFFFFFF ? -1 : i;
+  {
+    float st = ST, sd = SD;
+    warp_sum2(st, sd);
+    if (lane == 0) {
+      sm.rm[0][warp] = RT;
+      sm.rs[0][warp] = st;
+      sm.rm[1][warp] = RD;
+      sm.rs[1][warp] = sd;
+    }
+    if (__any_sync(0xffffffffu, badT) && lane == 0) atomicOr(&sm.flag, 1);
+    if (__any_sync(0xffffffffu, badD) && lane == 0) atomicOr(&sm.flag, 2);
+  }
+}
+
+// Pass 2 (L2): p and q per entry from the rows' lse (exponents LT, LD in
+// log2 units), TV, and the block masses of the row's draw (mode 1 residual,
+// 2 target), scored per block; the warp's TV and best block go to shared memory.
+template <typename TIn>
+__device__ __noinline__ void verify_pass2(VSmem& sm, const TIn* rT, const TIn* rD, int V, int nt,
+                                          bool hasD, int mode, bool badTr, bool badDr, float cT,
+                                          float LT, float LD, bool vec, uint64_t drop,
+                                          const Stream& sblk, uint32_t rid) {
+  constexpr int kUnroll = sizeof(TIn) == 2 ? 2 : 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float tvp = 0.f;
+  Cand best = cand_empty();
+  int nbuf = 0;
+  auto score_blocks = [&]() {
+    __syncwarp();
+    const int q = lane >> 1, h = lane & 1;  // lane: block h of buffered tile q
+    if (q < nbuf) {
+      float m = 0.f, e = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m += sm.part[warp][q][16 * h + i];
+      if (mode == 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) e += sm.pq[warp][q][16 * h + i];
+        e = 7.7e-6f * e + 1e-35f;  // |fp32 r - r| <= 7.7e-6 (p + q) per entry
+      }
+      const int jb = 2 * sm.tile[warp][q] + h;
+      if (m + e > 0.f) {
+        const U4 w = sblk.at((uint32_t)(jb >> 2), rid);
+        const float g32 = gumbel_f32(uniform_f32(word_of(w, jb & 3)));
+        Cand c;
+        if (mode == 1) {
+          const float lh = logf(m + e), lm = m > 0.f ? logf(m) : -INFINITY;
+          const float d = score_err(lh, g32);
+          c.s = lm + g32;
+          c.hi = lh + g32 + d;
+          c.lo = m - e > 0.f ? logf(m - e) + g32 - d : -INFINITY;
+        } else {
+          // the target's block mass from exps with arguments rounded in fp32
+          // (2^-24 of |z c| and of |lse log2 e|), ex2.approx and the sum
+          const float lm = logf(m);
+          const float d = score_err(lm, g32) + 2e-5f + 2e-7f * fabsf(LT);
+          c.s = lm + g32;
+          c.lo = c.s - d;
+          c.hi = c.s + d;
+        }
+        c.ohi = -INFINITY;
+        c.idx = jb;
+        c.aux = -1;
+        c.pad1 = c.pad2 = 0;
+        best = cand_merge(best, c);
+      }
+    }
+    __syncwarp();
+    nbuf = 0;
+  };
+  if (hasD || mode == 2) {
+    for (int t0 = warp; t0 < nt; t0 += kUnroll * kVWarps) {
+      Raw8<TIn> xt[kUnroll], xd[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int t = t0 + u * kVWarps;
+        if (t < nt) {
+          xt[u] = load8_raw<TIn>(rT, t * 256 + 8 * lane, V, vec, drop);
+          if (hasD) xd[u] = load8_raw<TIn>(rD, t * 256 + 8 * lane, V, vec, drop);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int t = t0 + u * kVWarps;
+        if (t >= nt) break;  // warp-uniform
+        float zt[8], zd[8];
+        unpack8<TIn>(xt[u], zt);
+        if (hasD) unpack8<TIn>(xd[u], zd);
+        float bm = 0.f, bpq = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float p = badTr ? 0.f : ex2(fmaf(zt[i], cT, -LT));
+          if (hasD) {
+            const float q = badDr ? 0.f : ex2(fmaf(zd[i], cT, -LD));
+            tvp += fabsf(p - q);
+            bm += fmaxf(p - q, 0.f);
+            bpq += p + q;
+          } else {
+            bm += p;
+          }
+        }
+        if (mode != 0) {
+          sm.part[warp][nbuf][lane] = bm;
+          if (mode == 1) sm.pq[warp][nbuf][lane] = bpq;
+          if (lane == 0) sm.tile[warp][nbuf] = t;
+          if (++nbuf == kVBuf) score_blocks();
+        }
+      }
+    }
+    if (mode != 0) score_blocks();
+  }
+  tvp = warp_sum(tvp);
+  best = warp_cand(best);
+  if (lane == 0) {
+    sm.tv[warp] = tvp;
+    sm.cand[warp] = best;
+  }
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(kVThreads, 1) verify_rows_kernel(const VerifyArgs a) {
-  using T8 = VT<TIn>;
-  constexpr int EPC = T8::EPC;
-  __shared__ VSmem sm;
-  const int tid = threadIdx.x;
-  const uint32_t rank = cluster_rank(), C = cluster_size();
-  const int j = (int)cluster_id();  // row unit: sequence b, position k
-  const int b = j / a.R, k = j % a.R;
-  const bool hasD = k < a.K;
-  const int s0 = (int)rank * a.slice;
-  const int len = max(0, min(a.slice, a.V - s0));
-  const TIn* rT = (const TIn*)a.zT + ((int64_t)b * a.R + k) * a.ld;
-  const TIn* rD = hasD ? (const TIn*)a.zD + ((int64_t)b * a.K + k) * a.ld : rT;
-  const TIn* gT = rT + s0;
-  const TIn* gD = rD + s0;
-  const bool vec = a.vec != 0;
+__global__ void __launch_bounds__(kVThreads, kVPerSM) verify_rows_kernel(const VerifyArgs a) {
+  extern __shared__ __align__(16) unsigned char vsmem[];
+  VSmem& sm = *reinterpret_cast<VSmem*>(vsmem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int V = a.V;
+  const int nt = (V + 255) / 256;
   const float cT = a.cT;
+  const bool vec = a.vec != 0;
+  const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
+  const int64_t nrows = (int64_t)a.B * a.R;
 
-  // ---------------- the row slices into registers
-  uint4 xT[kVChunks], xD[kVChunks];
-#pragma unroll
-  for (int c = 0; c < kVChunks; ++c) {
-    const int e0 = (tid + c * kVThreads) * EPC;
-    xT[c] = T8::load(gT, e0, len, vec);
-    xD[c] = hasD ? T8::load(gD, e0, len, vec) : xT[c];
-  }
-  const int x = hasD ? a.draft[(int64_t)b * a.K + k] : -1;
-  const bool x_ok = hasD && x >= 0 && x < a.V;
+  for (int64_t j = blockIdx.x; j < nrows; j += gridDim.x) {
+    const int b = (int)(j / a.R), k = (int)(j % a.R);
+    const bool hasD = k < a.K;
+    const TIn* rT = (const TIn*)a.zT + j * a.ld;
+    const TIn* rD = hasD ? (const TIn*)a.zD + ((int64_t)b * a.K + k) * a.ld : rT;
+    if (tid == 0) sm.flag = 0;
+    __syncthreads();
 
-  // ---------------- CTA maxima, then sums of exps relative to them
-  float mt = -INFINITY, md = -INFINITY;
+    verify_pass1<TIn>(sm, rT, rD, V, nt, hasD, cT, vec, keep);
+    __syncthreads();
+    if (warp == 0) {  // lse of both rows (fp64 combine): half-warp 0 the target, 1 the draft
+      const int h = lane >> 4, w = lane & 15;
+      const float pm = w < kVWarps ? sm.rm[h][w] : -INFINITY, ps = w < kVWarps ? sm.rs[h][w] : 0.f;
+      float MM = pm;
 #pragma unroll
-  for (int c = 0; c < kVChunks; ++c)
+      for (int o = 8; o > 0; o >>= 1) MM = fmaxf(MM, __shfl_xor_sync(0xffffffffu, MM, o));
+      double t = pm > -INFINITY ? (double)ps * (double)ex2((pm - MM) * cT) : 0.0;
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) {
-      mt = fmax_nan(mt, T8::get(xT[c], e));
-      md = fmax_nan(md, T8::get(xD[c], e));
-    }
-  const float4 mx = cta_max4_nan(make_float4(mt, md, 0.f, 0.f), &sm);
-  const float MtC = mx.x == -INFINITY ? 0.f : mx.x, MdC = mx.y == -INFINITY ? 0.f : mx.y;
-  const float nT = -MtC * cT, nD = -MdC * cT;
-  float st = 0.f, sd = 0.f;
-#pragma unroll
-  for (int c = 0; c < kVChunks; ++c)
-#pragma unroll
-    for (int e = 0; e < EPC; ++e) {
-      st += ex2(fmaf(T8::get(xT[c], e), cT, nT));
-      sd += ex2(fmaf(T8::get(xD[c], e), cT, nD));
-    }
-  const float4 sums = cta_sum4(make_float4(st, sd, 0.f, 0.f), &sm);
-  if (tid == 0) {
-    sm.ex.mT = mx.x;
-    sm.ex.sT = sums.x;
-    sm.ex.mD = mx.y;
-    sm.ex.sD = sums.y;
-    sm.ex.own = x_ok && x >= s0 && x < s0 + len;
-    if (sm.ex.own) {
-      sm.ex.zxT = Elem<TIn>::get(rT, x);
-      sm.ex.zxD = Elem<TIn>::get(rD, x);
-    }
-  }
-  // ---------------- the row's normalisers from every CTA of the cluster
-  cluster_sync();
-  float MT, ST, MD, SD, zxT = 0.f, zxD = 0.f;
-  double lseT, lseD;
-  {
-    const int lane = tid & 31;
-    const bool has = lane < (int)C;
-    float pm1 = -INFINITY, ps1 = 0.f, pm2 = -INFINITY, ps2 = 0.f;
-    int own = 0;
-    float zt = 0.f, zd = 0.f;
-    if (has) {
-      const uint32_t base = peer_addr(&sm.ex, (uint32_t)lane);
-      pm1 = ld_peer_f32(base + offsetof(VExch, mT));
-      ps1 = ld_peer_f32(base + offsetof(VExch, sT));
-      pm2 = ld_peer_f32(base + offsetof(VExch, mD));
-      ps2 = ld_peer_f32(base + offsetof(VExch, sD));
-      own = ld_peer_s32(base + offsetof(VExch, own));
-      if (own) {
-        zt = ld_peer_f32(base + offsetof(VExch, zxT));
-        zd = ld_peer_f32(base + offsetof(VExch, zxD));
+      for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      const double lse = (double)MM / a.tau64 + log(t);
+      if (w == 0) {
+        sm.lse[h] = lse;
+        if (!(MM > -INFINITY) && (h == 0 || hasD)) atomicOr(&sm.flag, h == 0 ? 1 : 2);
       }
-    }
-    float m1 = pm1, m2 = pm2;
-    warp_max2_nan(m1, m2);
-    MT = m1;
-    MD = m2;
-    float t1 = part_term(pm1, ps1, MT, cT), t2 = part_term(pm2, ps2, MD, cT);
-    warp_sum2(t1, t2);
-    ST = t1;
-    SD = t2;
-    const unsigned ob = __ballot_sync(0xffffffffu, own != 0);
-    if (ob) {
-      zxT = __shfl_sync(0xffffffffu, zt, __ffs(ob) - 1);
-      zxD = __shfl_sync(0xffffffffu, zd, __ffs(ob) - 1);
-    }
-    // fp64 log-sum-exp: the slice factors in fp32, their sums and the log in fp64
-    double d1 = (has && pm1 > -INFINITY) ? (double)ps1 * (double)ex2((pm1 - MT) * cT) : 0.0;
-    double d2 = (has && pm2 > -INFINITY) ? (double)ps2 * (double)ex2((pm2 - MD) * cT) : 0.0;
-    d1 = warp_sum_d(d1);
-    d2 = warp_sum_d(d2);
-    lseT = (double)MT / a.tau64 + log(d1);
-    lseD = (double)MD / a.tau64 + log(d2);
-  }
-  const bool badT = !(MT > -INFINITY && MT < INFINITY && ST > 0.f && ST < INFINITY);
-  const bool badD = hasD && !(MD > -INFINITY && MD < INFINITY && SD > 0.f && SD < INFINITY);
-  const bool bad = badT || badD;
-
-  // ---------------- the accept test (every CTA of the row takes it alike)
-  bool accept = false;
-  if (hasD && !bad && x_ok) {
-    const double p = exp((double)zxT / a.tau64 - lseT);
-    const double q = exp((double)zxD / a.tau64 - lseD);
-    const Stream sa(a.seed, a.round, SD_STREAM_ACCEPT);
-    const double u = uniform_f64(sa.at(0, (uint32_t)j).x);
-    accept = u * q < p;
-  }
-
-  // ---------------- TV, and the draw this row needs
-  // per-thread scale factors turning the CTA-relative exps into probabilities
-  const float scT = (!badT && mx.x > -INFINITY) ? ex2((MtC - MT) * cT) / ST : 0.f;
-  const float scD = (hasD && !badD && mx.y > -INFINITY) ? ex2((MdC - MD) * cT) / SD : 0.f;
-  const bool draw_resid = hasD && !bad && !accept;
-  const bool draw_bonus = !hasD && !badT;
-  const Stream sr(a.seed, a.round, draw_resid ? SD_STREAM_RESIDUAL : SD_STREAM_BONUS);
-  const uint32_t rowid = draw_resid ? (uint32_t)j : (uint32_t)b;
-  float tvp = 0.f;
-  Cand best = cand_empty();
-  if (hasD && !draw_resid) {
-#pragma unroll
-    for (int c = 0; c < kVChunks; ++c)
-#pragma unroll
-      for (int e = 0; e < EPC; ++e) {
-        const float p = ex2(fmaf(T8::get(xT[c], e), cT, nT)) * scT;
-        const float q = ex2(fmaf(T8::get(xD[c], e), cT, nD)) * scD;
-        tvp += fabsf(p - q);
-      }
-  } else if (draw_resid) {
-    // TV and the residual screen in one pass.  Tr, a lower bound on the
-    // winner's score, is the best fp32 lower bound among the entries this thread
-    // has scored so far (any entry's score bounds the winner's from below; -inf
-    // at first).  With y = (r + eb) e^{-Tr}, u <= 1 - y proves log r + g <= Tr
-    // (e^{-y} >= 1 - y): the entry cannot win and takes no log; four entries
-    // whose y all stay below e^{-g_max} skip the Philox call.
-    float Tr = -INFINITY, eTr = INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < kVChunks; ++c) {
-#pragma unroll 1
-      for (int h = 0; h < EPC / 4; ++h) {
-        float r4[4], eb4[4], ymax = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float zt = T8::get(xT[c], 4 * h + e), zd = T8::get(xD[c], 4 * h + e);
-          const float p = ex2(fmaf(zt, cT, nT)) * scT, q = ex2(fmaf(zd, cT, nD)) * scD;
-          tvp += fabsf(p - q);
-          r4[e] = p - q;
-          eb4[e] = 7.7e-6f * (p + q) + 1e-37f;
-          ymax = fmaxf(ymax, (r4[e] + eb4[e]) * eTr);
-        }
-        const int v0 = s0 + (tid + c * kVThreads) * EPC + 4 * h;
-        if (!(ymax >= kYSkip) || v0 >= s0 + len) continue;
-        const U4 w = sr.at((uint32_t)(v0 >> 2), rowid);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float ub = r4[e] + eb4[e];
-          if (!(ub > 0.f) || v0 + e >= s0 + len) continue;
-          const float u = uniform_f32(word_of(w, e));
-          if (Tr > -INFINITY && !keep_bonus(ub * eTr, u)) continue;
-          const float g32 = gumbel_f32(u);
-          const float hl = logf(ub);
-          const float d = score_err(hl, g32);
-          Cand cd;
-          cd.hi = hl + g32 + d;
-          if (!(cd.hi >= Tr)) continue;
-          cd.s = r4[e] > 0.f ? logf(r4[e]) + g32 : -INFINITY;
-          cd.lo = r4[e] - eb4[e] > 0.f ? logf(r4[e] - eb4[e]) + g32 - d : -INFINITY;
-          cd.ohi = -INFINITY;
-          cd.idx = v0 + e;
-          cd.aux = -1;
-          cd.pad1 = cd.pad2 = 0;
-          best = cand_merge(best, cd);
-          if (cd.lo > Tr) {
-            Tr = cd.lo;
-            eTr = ex2(-Tr * kLog2e) * 1.001f;  // (rounded up: keeps the tests conservative)
-          }
+      __syncwarp();
+      if (lane == 0 && hasD && !(sm.flag & 3)) {  // the accept test, fp64
+        const int x = a.draft[(int64_t)b * a.K + k];
+        if (x >= 0 && x < V) {
+          const double p = exp((double)ld_elem<TIn>(rT, x) / a.tau64 - sm.lse[0]);
+          const double q = exp((double)ld_elem<TIn>(rD, x) / a.tau64 - sm.lse[1]);
+          const Stream sa(a.seed, a.round, SD_STREAM_ACCEPT);
+          const double uu = uniform_f64(sa.at(0, (uint32_t)j).x);
+          if (uu * q < p) atomicOr(&sm.flag, 4);
+        } else {
+          atomicOr(&sm.flag, 8);
         }
       }
     }
-  } else if (draw_bonus) {
-    // T = M/tau + g_min - margin bounds the winning score from below; an entry
-    // whose uniform proves u <= 1 - e^{a - T} cannot win (integer leading-bit
-    // test first), four entries that even g_max cannot lift to T skip Philox.
-    const float aM = MT * a.inv_tau;
-    const float Tc = (aM + kGumbelMinF - (1e-5f + 2e-7f * fabsf(aM))) * kLog2e;
-#pragma unroll 1
-    for (int c = 0; c < kVChunks; ++c) {
-#pragma unroll 1
-      for (int h = 0; h < EPC / 4; ++h) {
-        float z4[4], X4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          z4[e] = T8::get(xT[c], 4 * h + e);
-          X4[e] = fmaf(z4[e], cT, -Tc);
-        }
-        if (!(fmaxf(fmaxf(X4[0], X4[1]), fmaxf(X4[2], X4[3])) > -24.05f)) continue;
-        const int v0 = s0 + (tid + c * kVThreads) * EPC + 4 * h;
-        const U4 w = sr.at((uint32_t)(v0 >> 2), rowid);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t wj = word_of(w, e);
-          const uint32_t Rr = 0x7FFFFFu - (wj >> 9);
-          const int hb = Rr ? 31 - __clz((int)Rr) : -1;
-          if (!(X4[e] > (float)(hb - 23) - 0.01f) || v0 + e >= s0 + len) continue;
-          const float u = uniform_f32(wj);
-          if (keep_bonus(ex2(X4[e]), u)) best = cand_merge(best, bonus_cand_a(z4[e] * a.inv_tau, u, v0 + e));
-        }
+    __syncthreads();
+    const int flag = sm.flag;
+    const bool badTr = (flag & 1) != 0, badDr = hasD && (flag & 2) != 0;
+    const bool bad = badTr || badDr;
+    const bool accept = (flag & 4) != 0;
+    const double lseT = sm.lse[0], lseD = sm.lse[1];
+    // the draw this row needs: 1 the residual (a rejection), 2 the bonus (the last row)
+    const int mode = bad ? 0 : (hasD ? (accept ? 0 : 1) : 2);
+
+    const float LT = (float)(lseT * 1.4426950408889634), LD = (float)(lseD * 1.4426950408889634);
+    const Stream sblk(a.seed, a.round, mode == 1 ? SD_STREAM_RESIDUAL_BLOCK : SD_STREAM_BONUS_BLOCK);
+    const uint32_t rid = mode == 1 ? (uint32_t)j : (uint32_t)b;
+    verify_pass2<TIn>(sm, rT, rD, V, nt, hasD, mode, badTr, badDr, cT, LT, LD, vec, drop, sblk, rid);
+    // ---------------- the row's TV and block
+    __syncthreads();
+    if (warp == 0) {
+      float tv = lane < kVWarps ? sm.tv[lane] : 0.f;
+      tv = warp_sum(tv);
+      Cand c = lane < kVWarps ? sm.cand[lane] : cand_empty();
+      c = warp_cand(c);
+      if (lane == 0) {
+        if (hasD && a.tv_out) a.tv_out[(int64_t)b * a.K + k] = bad ? NAN : 0.5f * tv;
+        // -2: no candidate; -1: settle in fp64; else the block
+        sm.block = c.idx == 0x7FFFFFFF ? -2 : (c.ohi < c.lo ? c.idx : -1);
       }
     }
-  }
-  // ---------------- the row's TV and candidates, gathered at the leader CTA
-  const float4 tvs = cta_sum4(make_float4(tvp, 0.f, 0.f, 0.f), &sm);
-  best = cta_cand(best, &sm);
-  if (tid == 0) {
-    sm.ex.tvp = tvs.x;
-    sm.ex.cand = best;
-  }
-  cluster_sync();
-  if (rank == 0 && tid < 32) {
-    const int lane = tid;
-    const bool has = lane < (int)C;
-    float tv = 0.f;
-    Cand cd = cand_empty();
-    if (has) {
-      const uint32_t base = peer_addr(&sm.ex, (uint32_t)lane);
-      tv = ld_peer_f32(base + offsetof(VExch, tvp));
-      cd.s = ld_peer_f32(base + offsetof(VExch, cand) + offsetof(Cand, s));
-      cd.lo = ld_peer_f32(base + offsetof(VExch, cand) + offsetof(Cand, lo));
-      cd.hi = ld_peer_f32(base + offsetof(VExch, cand) + offsetof(Cand, hi));
-      cd.ohi = ld_peer_f32(base + offsetof(VExch, cand) + offsetof(Cand, ohi));
-      cd.idx = ld_peer_s32(base + offsetof(VExch, cand) + offsetof(Cand, idx));
-    }
-    tv = warp_sum(tv);
-    cd = warp_cand(cd);
-    if (lane == 0) {
-      if (hasD && a.tv_out) a.tv_out[(int64_t)b * a.K + k] = bad ? NAN : 0.5f * tv;
-      sm.wc[0] = cd;
-    }
-  }
-  cluster_sync();  // every CTA's exchange slot has been read: peers may finish
-  if (rank != 0) return;
-
-  // ---------------- the leader encodes the row's outcome
-  int code;
-  if (hasD) {
-    if (bad) {
-      code = kCodeBad;
-      if (tid == 0) raise_err(a.dev_err, SD_DEV_NONFINITE);
-    } else if (accept) {
-      code = x;
-    } else {
-      const Cand cd = sm.wc[0];
-      int tok;
+    __syncthreads();
+    int code = kCodeBad;
+    if (mode != 0) {
+      int dmode = mode;  // 1 residual, 2 bonus, 0 target after a zero residual
       bool zr = false;
-      if (cd.idx == 0x7FFFFFFF) {  // no residual mass in fp32: decide exactly
-        tok = exact_draw_row<TIn>(rT, rD, a.V, 1, lseT, lseD, a, -INFINITY, sr, rowid, &sm);
-        if (tok < 0) {  // the exact residual is zero everywhere: draw from p
+      int jb = sm.block;
+      const Stream sb_res(a.seed, a.round, SD_STREAM_RESIDUAL_BLOCK);
+      if (jb < 0) {
+        jb = exact_block<TIn>(sm, rT, rD, V, dmode, a.tau64, lseT, lseD, sblk, rid);
+        if (jb < 0 && mode == 1) {  // the exact residual is zero everywhere: draw from p
           zr = true;
-          tok = exact_draw_row<TIn>(rT, rD, a.V, 0, lseT, lseD, a, -INFINITY, sr, rowid, &sm);
+          dmode = 0;
+          jb = exact_block<TIn>(sm, rT, rD, V, 0, a.tau64, lseT, lseD, sb_res, rid);
         }
-      } else if (cd.ohi < cd.lo) {
-        tok = cd.idx;
-      } else {  // near-tie: exact fp64 re-score of every entry that can still win
-        tok = exact_draw_row<TIn>(rT, rD, a.V, 1, lseT, lseD, a, cd.lo, sr, rowid, &sm);
       }
-      code = encode_reject(max(tok, 0), !x_ok, zr);
+      if (warp == 0) {
+        const Stream se(a.seed, a.round, mode == 1 ? SD_STREAM_RESIDUAL : SD_STREAM_BONUS);
+        const int tok = jb >= 0 ? exact_in_block<TIn>(rT, rD, V, jb, dmode, a.tau64, lseT, lseD, se, rid) : -1;
+        if (mode == 1) code = encode_reject(max(tok, 0), (flag & 8) != 0, zr);
+        else code = tok;
+      }
+    } else if (hasD && !bad) {
+      code = a.draft[(int64_t)b * a.K + k];  // accepted
     }
-  } else {
-    if (badT) {
-      code = kCodeBad;
-    } else {
-      const Cand cd = sm.wc[0];
-      if (cd.idx == 0x7FFFFFFF) code = -1;
-      else if (cd.ohi < cd.lo) code = cd.idx;
-      else code = exact_draw_row<TIn>(rT, rT, a.V, 0, lseT, lseD, a, cd.lo, sr, rowid, &sm);
+    if (tid == 0) {
+      if (hasD && bad) raise_err(a.dev_err, SD_DEV_NONFINITE);
+      a.out_tokens[j] = code;
     }
+    __syncthreads();  // shared state is reused by the next row
   }
-  if (tid == 0) a.out_tokens[(int64_t)b * a.R + k] = code;
 }
 
 // Per sequence: the first rejection (or the end) decides the accepted length
@@ -539,18 +474,22 @@ __global__ void verify_finalize_kernel(int B, int K, int32_t* out_tokens, int32_
 
 template <typename TIn>
 static sd_status launch_verify(VerifyArgs& a, int B, cudaStream_t stream) {
-  a.slice = kVThreads * kVChunks * VT<TIn>::EPC;
-  const int C = (a.V + a.slice - 1) / a.slice;
-  if (C > kMaxCluster) return SD_ERR_UNSUPPORTED;
-  a.slice = ((a.V + C - 1) / C + 7) / 8 * 8;  // balanced slices (multiples of 8 entries)
-  const void* fn = (const void*)verify_rows_kernel<TIn>;
-  if (C > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+  int dev = 0, nsm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     cudaGetLastError();
     return SD_ERR_CUDA;
   }
-  LaunchPlan p{C, 1, kVThreads, 0, a.slice, 0, 0, 0};
-  const sd_status st = launch_clusters(fn, p, (int64_t)B * a.R, a, stream);
-  if (st != SD_OK) return st;
+  const int64_t rows = (int64_t)B * a.R;
+  const int grid = (int)(rows < kVPerSM * nsm ? rows : kVPerSM * nsm);  // persistent CTAs
+  const int smem = (int)sizeof(VSmem);
+  const void* fn = (const void*)verify_rows_kernel<TIn>;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return SD_ERR_CUDA;
+  }
+  verify_rows_kernel<TIn><<<grid, kVThreads, smem, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
   verify_finalize_kernel<<<(B + 127) / 128, 128, 0, stream>>>(B, a.K, a.out_tokens, a.acc_len,
                                                                a.dev_err);
   if (cudaGetLastError() != cudaSuccess) return SD_ERR_CUDA;
@@ -576,6 +515,7 @@ extern "C" sd_status sd_verify_reject(const void* zT, const void* zD, sd_dtype d
   a.zT = zT;
   a.zD = zD;
   a.ld = ld;
+  a.B = B;
   a.V = V;
   a.K = K;
   a.R = K + 1;

@@ -21,7 +21,7 @@
 //            observations in batch order: old entries on lanes 0..k-1, the
 //            observation on lanes k..2k-1, partners found by __match_any_sync,
 //            values (c * old + obs) / (c + 1) in fp64 with one rounding per
-//            operation, and the new top k by rank counting across the warp;
+//            operation, and the new top k by a bitonic sort across the warp;
 //   lookup   one warp per query probes the same way and copies the row out.
 //
 // Table layout in one caller-owned device buffer (capacity C, a power of two,
@@ -423,8 +423,6 @@ constexpr int kMergeThreads = 256;
 __global__ void __launch_bounds__(kMergeThreads) ngram_merge_kernel(
     TableView t, const int32_t* __restrict__ ctx, int n, const int32_t* __restrict__ idx,
     const float* __restrict__ prob, int U, const int32_t* __restrict__ ws, uint32_t* dev_err) {
-  __shared__ int st_i[kMergeThreads / 32][32];
-  __shared__ float st_p[kMergeThreads / 32][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int k = t.k;
   const int D = min(max(ws[0], 0), U), W = min(max(ws[1], 0), U);
@@ -455,13 +453,21 @@ __global__ void __launch_bounds__(kMergeThreads) ngram_merge_kernel(
         op = t.prob[slot * k + lane];
       }
     }
+    // the next observation's row is loaded while this one merges
+    int nxi = -1;
+    float nxp = 0.f;
+    if (is_obs) {
+      const int u0 = perm[q0];
+      nxi = idx[(int64_t)u0 * k + (lane - k)];
+      nxp = prob[(int64_t)u0 * k + (lane - k)];
+    }
     for (int q = q0; q < q1; ++q) {
-      const int u = perm[q];
-      int xi = -1;
-      float xp = 0.f;
-      if (is_obs) {
-        xi = idx[(int64_t)u * k + (lane - k)];
-        xp = prob[(int64_t)u * k + (lane - k)];
+      const int xi = nxi;
+      const float xp = nxp;
+      if (is_obs && q + 1 < q1) {
+        const int un = perm[q + 1];
+        nxi = idx[(int64_t)un * k + (lane - k)];
+        nxp = prob[(int64_t)un * k + (lane - k)];
       }
       // one id per lane for matching; empty entries get ids no other lane has
       const int id = is_old ? (oi >= 0 ? oi : -2 - lane) : (is_obs && xi >= 0 ? xi : -2 - lane);
@@ -490,25 +496,29 @@ __global__ void __launch_bounds__(kMergeThreads) ngram_merge_kernel(
         const double num = __dadd_rn(__dmul_rn(cd, 0.0), (double)xp);
         val = __double2float_rn(__ddiv_rn(num, cd + 1.0));
       }
-      // rank in (value descending, index ascending) order among the candidates
-      const unsigned cmask = __ballot_sync(0xffffffffu, cand);
-      int rank = 0;
-      for (int j = 0; j < 32; ++j) {
-        const float vj = __shfl_sync(0xffffffffu, val, j);
-        const int ij = __shfl_sync(0xffffffffu, vid, j);
-        if (((cmask >> j) & 1u) && (vj > val || (vj == val && ij < vid))) ++rank;
+      // bitonic sort of the warp's lanes in (value descending, index
+      // ascending) order, non-candidates last: lane r ends with rank r
+      const int ncand = __popc(__ballot_sync(0xffffffffu, cand));
+      float sv = cand ? val : -INFINITY;
+      int si = cand ? vid : 0x7FFFFFFF;
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, sv, stride);
+          const int oi2 = __shfl_xor_sync(0xffffffffu, si, stride);
+          const bool other_first = ov > sv || (ov == sv && oi2 < si);
+          const bool lower = (lane & stride) == 0, up = (lane & size) == 0;
+          if (lower == up ? other_first : !other_first && (ov != sv || oi2 != si)) {
+            sv = ov;
+            si = oi2;
+          }
+        }
       }
-      if (cand && rank < k) {
-        st_i[warp][rank] = vid;
-        st_p[warp][rank] = val;
-      }
-      __syncwarp();
-      const int ncand = __popc(cmask);
       if (is_old) {
-        oi = lane < ncand ? st_i[warp][lane] : -1;
-        op = lane < ncand ? st_p[warp][lane] : 0.f;
+        oi = lane < ncand ? si : -1;
+        op = lane < ncand ? sv : 0.f;
       }
-      __syncwarp();
       ++c;
     }
     if (is_old) {

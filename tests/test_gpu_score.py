@@ -153,6 +153,37 @@ def test_identical_rows_invariants():
     assert np.all(g["tv"] == 0.0)
 
 
+def test_ragged_vocab_padded_stride():
+    """V not a multiple of the 8-entry chunk, rows padded to a 16-byte stride:
+    the last chunk of every row is read entry by entry."""
+    rng = np.random.default_rng(16)
+    V = 33001
+    zT, zD, x = rand_case(rng, 2, 5, 3, V)
+    g = run_score(zT, zD, x, 0.9, 21, 2, ld=33008)
+    o = oracle.smcsd_score(zT, zD, x, 0.9, 21, 2)
+    compare(g, o, "ragged_padded")
+
+
+def test_without_tv_output():
+    """tv_out = NULL: the other outputs are unchanged."""
+    rng = np.random.default_rng(17)
+    B, N, K, V = 2, 6, 3, 40960
+    zT, zD, x = rand_case(rng, B, N, K, V)
+    g = run_score(zT, zD, x, 1.0, 5, 8)
+    t, d = bf16_dev(zT), bf16_dev(zD)
+    xs = to_dev(x)
+    logw = torch.empty((B, N), dtype=torch.float64, device="cuda")
+    bonus = torch.empty((B, N), dtype=torch.int32, device="cuda")
+    lse = torch.empty((B, N, K + 1, 2), dtype=torch.float64, device="cuda")
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    lib.smcsd_score(t, d, xs, 1.0, 5, 8, logw, bonus, lse_out=lse, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(logw.cpu().numpy(), g["logw"])
+    assert np.array_equal(bonus.cpu().numpy(), g["bonus"])
+    assert np.array_equal(lse.cpu().numpy(), g["lse"])
+
+
 def test_faults_set_error_bits():
     rng = np.random.default_rng(14)
     zT, zD, x = rand_case(rng, 1, 3, 2, 2000)

@@ -18,18 +18,20 @@ namespace smcsd {
 //     row's slices from the ring to registers, warp maxima, exps (one MUFU
 //     exp2 per entry) and sums; the exps of both halves go to tensor memory
 //     (TMEM, two row buffers per warp); post the (max, sum) partials.
-//     On a particle's last row they also sum the target exps of each
-//     128-entry block and post the best block candidate of the bonus draw
-//     (a two-level Gumbel-max: the block by log-mass plus block noise, then
-//     the entry inside it).
+//     On a particle's last row they also park each lane's chunk sums of the
+//     target exps for the bonus draw (a two-level Gumbel-max: the block by
+//     log-mass plus block noise, then the entry inside it); fp32 rows post
+//     their warp's best block candidate instead.
 //   consumers (four, one per TMEM lane quarter), one row behind: once the
 //     row's messages are in, rebuild its normalisers, read the exps back from
 //     TMEM and take the TV partial sum |p - q|; then hand the row buffer back.
 //   communication: turns the producers' partials into one 32-byte message per
 //     row for every CTA of the cluster (st.async into distributed shared
 //     memory, completing on the receiver's mbarrier -- no cluster barrier on
-//     the row path), sends each row's TV partial and bonus candidate to the
-//     leader, and refills the ring with bulk async copies (no multicast).
+//     the row path), scores a last row's 128-entry blocks from the parked
+//     sums once its message is out (off the producers' path), sends each
+//     row's TV partial and bonus candidate to the leader, and refills the
+//     ring with bulk async copies (no multicast).
 //   bookkeeping (leader only): fp64 lse, log-probs, log-weights, TV and bonus
 //     tokens: the block from the candidates (a near-tie in fp64 over the
 //     row's blocks), then the entry inside it from its 128 logits.
@@ -45,6 +47,10 @@ constexpr int kConsumers = 4;        // phase-B warps, one per TMEM lane quarter
 constexpr int kMaxThreadsSmc = 640;  // up to 14 producers + 4 consumers + 2 service warps
 static_assert(kMaxThreadsSmc / 32 - kConsumers - 2 <= 16, "one lane per producer in each half-warp");
 constexpr size_t kMinSmem = 120 * 1024;  // > half an SM's shared memory: one CTA per SM
+// bf16 rows: producers park each lane's chunk sums of a particle's last row
+// (by row & 3, [warp][chunk][lane]) for the communication warp's block scores.
+constexpr int kBpartRows = 4;
+constexpr size_t kBpartBytes = (size_t)kBpartRows * kMaxWarps * (kEPT / 8) * 32 * sizeof(float);
 
 struct alignas(16) BMsg {  // one slice's phase-B results for the leader
   float tv, s, lo, hi;
@@ -426,6 +432,7 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
   const int nS = a.stages;
   const size_t sb = a.stage_bytes;  // one tensor's slice; a stage holds both
   SmcTail* tl = reinterpret_cast<SmcTail*>(smem + (size_t)nS * 2 * sb);
+  float* bpart = reinterpret_cast<float*>(smem + (size_t)nS * 2 * sb + sizeof(SmcTail));
 
   const int s0 = (int)rank * a.slice;
   const int len = max(0, min(a.slice, a.V - s0));
@@ -485,6 +492,9 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
     if (lane == 0)
       for (int i = 0; i < nS && i < nrows; ++i) issue(i, i);
     int k = 0, stage = 0;  // position and ring stage of row it
+    float mwT_row = -INFINITY;   // lane w: producer warp w's target maximum of row it
+    Cand pend = cand_empty();    // bf16: bonus candidate of the last row whose message went out
+    const Stream blkst(a.seed, a.round, SD_STREAM_BONUS_BLOCK);
     for (int it = 0; it <= nrows; ++it) {
       if (it < nrows) {  // row it: refill its stage once read, then its message
         if (it + nS < nrows) {
@@ -494,6 +504,7 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
         swait(&tl->afull[it & 1], (uint32_t)((it >> 1) & 1), tl, a.dev_err, kWsAfull);
         const float4 wp =
             lane < nA ? tl->wpart[it & 1][lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        mwT_row = wp.x;
         float mT = wp.x, mD = wp.z;
         warp_max2_nan(mT, mD);  // a warp's NaN max (NaN in its entries) must reach the sum
         float sumT = part_term(wp.x, wp.y, mT, cT), sumD = part_term(wp.z, wp.w, mD, cT);
@@ -526,9 +537,13 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
         tv = warp_sum(tv);
         const int pk = k == 0 ? a.R - 1 : k - 1;
         Cand cd = cand_empty();
-        if (pk == a.K) {  // the producers posted its bonus blocks with the row
-          if (lane < nA) cd = tl->wcand[p & 3][lane];
-          cd = warp_cand(cd);
+        if (pk == a.K) {
+          if (EPC == 8) {
+            cd = pend;  // scored by this warp after the row's message
+          } else {  // the producers posted its bonus blocks with the row
+            if (lane < nA) cd = tl->wcand[p & 3][lane];
+            cd = warp_cand(cd);
+          }
         }
         const int pslot = p % kRing;
         if (leader && lane == 0) mbar_arrive_expect_tx(&tl->bbar[pslot], C * (uint32_t)sizeof(BMsg));
@@ -538,6 +553,49 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
           st_async_v4(ra, want_tv ? tv : 0.f, cd.s, cd.lo, cd.hi, rb);
           st_async_v4(ra + 16, cd.ohi, __int_as_float(cd.idx), 0.f, 0.f, rb);
         }
+      }
+      if (EPC == 8 && it < nrows && k == a.K) {
+        // Row it's bonus blocks from the lanes' parked chunk sums: block (w, c, h)
+        // is lanes 16h..16h+15 of warp w's chunk row c, local entries
+        // 256 (c nA + w) + 128 h; lambda = ln(sum) + m_w / tau (the exps are
+        // relative to the warp's maximum m_w) plus the block's noise, with fp32
+        // error bounds.  A block whose exps all flushed to 0 lies > 80 nats below
+        // its warp's best block and cannot win (block noise spans < 20).
+        const float* bp = bpart + (size_t)(it & (kBpartRows - 1)) * kMaxWarps * CPT * 32;
+        const int64_t unit = (int64_t)cid + (int64_t)(it / a.R) * G;
+        const int nlb = 2 * CPT * nA;
+        Cand cd = cand_empty();
+        for (int lb0 = 0; lb0 < nlb; lb0 += 32) {  // warp-uniform trip count (shuffles)
+          const int lb = lb0 + lane;
+          const int c = lb / (2 * nA), w = (lb >> 1) % nA, h = lb & 1;
+          const int local = 256 * (c * nA + w) + 128 * h;
+          const float mw = __shfl_sync(0xffffffffu, mwT_row, w);
+          if (lb < nlb && local < len) {
+            const float4* q = reinterpret_cast<const float4*>(bp + (w * CPT + c) * 32 + 16 * h);
+            const float4 q0 = q[0], q1 = q[1], q2 = q[2], q3 = q[3];
+            const float sum = ((q0.x + q0.y) + (q0.z + q0.w)) + ((q1.x + q1.y) + (q1.z + q1.w)) +
+                              ((q2.x + q2.y) + (q2.z + q2.w)) + ((q3.x + q3.y) + (q3.z + q3.w));
+            if (sum > 0.f) {
+              const float mws = mw == -INFINITY ? 0.f : mw;
+              const int jb = (s0 + local) / kBlk;
+              const U4 wr = blkst.at((uint32_t)(jb >> 2), (uint32_t)unit);
+              const float g32 = gumbel_f32(uniform_f32(word_of(wr, jb & 3)));
+              const float lam = logf(sum) + mws * a.inv_tau;
+              const float sc = lam + g32;
+              const float d = score_err(lam, g32) + 2e-5f + 2e-7f * fabsf(mws * cT);
+              Cand e;
+              e.s = sc;
+              e.lo = sc - d;
+              e.hi = sc + d;
+              e.ohi = -INFINITY;
+              e.idx = jb;
+              e.aux = -1;
+              e.pad1 = e.pad2 = 0;
+              cd = cand_merge(cd, e);
+            }
+          }
+        }
+        pend = warp_cand(cd);
       }
       if (it < nrows && ++k == a.R) k = 0;
     }
@@ -726,7 +784,10 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
       }
       accT = __fadd2_rn(accT, bacc);
       accD = __fadd2_rn(accD, dacc);
-      if (brow) {  // a chunk row of the warp is one block (fp32) or two (bf16: half-warps)
+      if (brow && EPC == 8) {  // bf16: the lane's chunk sum, scored by the communication warp
+        bpart[(size_t)(it & (kBpartRows - 1)) * kMaxWarps * CPT * 32 + (warp * CPT + c) * 32 + lane] =
+            bacc.x + bacc.y;
+      } else if (brow) {  // fp32: a chunk row of the warp is one block
         float sb = bacc.x + bacc.y;
         if (EPC == 8) {
 #pragma unroll
@@ -741,7 +802,7 @@ __global__ void __launch_bounds__(kMaxThreadsSmc, 1) smc_kernel(const ScoreArgs 
         }
       }
     }
-    if (brow) {
+    if (brow && EPC != 8) {
       // Block candidates of the bonus draw: lambda_j = ln(sum) + m/tau (the exps
       // are relative to the warp max m) plus the block's Gumbel noise, with fp32
       // error bounds.  A block whose exps all flushed to 0 lies > 80 nats below
@@ -826,14 +887,15 @@ static bool make_plan_smc(const void* fn, int V, int esize, int64_t units, Launc
     const int threads = ncomp + 32 * (kConsumers + 2);  // + consumers, communication, bookkeeping
     if (threads > kMaxThreadsSmc || ncomp / 32 > kMaxWarps) continue;
     const uint32_t sb = (uint32_t)(((int64_t)slice * esize + 127) / 128 * 128);
+    const size_t extra = esize == 2 ? kBpartBytes : 0;  // parked bonus chunk sums (bf16)
     int nS = 0;
     for (int st = kMaxStages; st >= 2; --st)
-      if ((size_t)st * 2 * sb + sizeof(SmcTail) + 128 <= (size_t)optin) {
+      if ((size_t)st * 2 * sb + sizeof(SmcTail) + extra + 128 <= (size_t)optin) {
         nS = st;
         break;
       }
     if (nS == 0) continue;
-    const size_t smem = std::max((size_t)nS * 2 * sb + sizeof(SmcTail) + 128, kMinSmem);
+    const size_t smem = std::max((size_t)nS * 2 * sb + sizeof(SmcTail) + extra + 128, kMinSmem);
     const int nc = max_active_clusters(fn, C, threads, smem);
     if (nc <= 0) continue;
     const int64_t score = std::min<int64_t>(ukey, nc) * C * 8 + nS;

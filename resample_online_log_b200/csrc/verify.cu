@@ -16,8 +16,9 @@
 //     in turn, streaming each row twice in tiles of 256 entries (8 per lane,
 //     16-byte loads, several tiles in flight):
 //     pass 1 (HBM; the row stays in L2): the log-sum-exp of the target and
-//       draft rows, exps relative to each warp's running max (one redux per
-//       tile); the accept test u q(x) < p(x) in fp64;
+//       draft rows, exps relative to each lane's running max (the warp
+//       combines its lanes once, after the row); the accept test
+//       u q(x) < p(x) in fp64;
 //     pass 2 (L2): p and q per entry, TV = 1/2 sum |p - q|, and the block
 //       masses the row's draw needs -- residual sum max(p - q, 0) after a
 //       rejection (with the error bound 7.7e-6 (p + q) per entry), target
@@ -151,15 +152,15 @@ __device__ __noinline__ int exact_in_block(const TIn* rT, const TIn* rD, int V, 
   return bi == 0x7FFFFFFF ? -1 : bi;
 }
 
-// Pass 1 over a row pair (HBM; the rows are left in L2 for pass 2): per warp
-// the target's and draft's running max and sums of exps relative to it, and
-// NaN / +inf flags, into shared memory.
+// Pass 1 over a row pair (HBM; the rows are left in L2 for pass 2): each lane
+// keeps its own running max and sum of exps relative to it for the target and
+// draft rows (no cross-lane step inside the loop), then the warp combines
+// them; the warp's (max, sum) pairs and NaN / +inf flags go to shared memory.
 template <typename TIn>
 __device__ __noinline__ void verify_pass1(VSmem& sm, const TIn* rT, const TIn* rD, int V, int nt,
                                           bool hasD, float cT, bool vec, uint64_t keep) {
   constexpr int kUnroll = sizeof(TIn) == 2 ? 2 : 1;  // tiles in flight per tensor (32 bytes a lane)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // ---------------- pass 1 (HBM): the two rows' log-sum-exp
   float RT = -INFINITY, RD = -INFINITY, ST = 0.f, SD = 0.f;
   bool badT = false, badD = false;
   for (int t0 = warp; t0 < nt; t0 += kUnroll * kVWarps) {
@@ -177,21 +178,9 @@ __device__ __noinline__ void verify_pass1(VSmem& sm, const TIn* rT, const TIn* r
       if (t0 + u * kVWarps >= nt) break;  // warp-uniform
       float zt[8], zd[8];
       unpack8<TIn>(xt[u], zt);
-      float mt = -INFINITY, md = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mt = fmax_nan(mt, zt[i]);
-      if (hasD) {
-        unpack8<TIn>(xd[u], zd);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) md = fmax_nan(md, zd[i]);
-      }
-      badT |= mt != mt;
-      badD |= md != md;
-      mt = mt != mt ? -INFINITY : mt;
-      md = md != md ? -INFINITY : md;
-      warp_max2(mt, md);
-      badT |= mt == INFINITY;
-      badD |= md == INFINITY;
+      float mt = fmax_nan(fmax_nan(fmax_nan(zt[0], zt[1]), fmax_nan(zt[2], zt[3])),
+                          fmax_nan(fmax_nan(zt[4], zt[5]), fmax_nan(zt[6], zt[7])));
+      badT |= mt != mt || mt == INFINITY;
       if (mt > RT) {
         ST = RT == -INFINITY ? 0.f : ST * ex2((RT - mt) * cT);
         RT = mt;
@@ -202,6 +191,10 @@ __device__ __noinline__ void verify_pass1(VSmem& sm, const TIn* rT, const TIn* r
         for (int i = 0; i < 8; ++i) ST += ex2(fmaf(zt[i], cT, n));
       }
       if (hasD) {
+        unpack8<TIn>(xd[u], zd);
+        float md = fmax_nan(fmax_nan(fmax_nan(zd[0], zd[1]), fmax_nan(zd[2], zd[3])),
+                            fmax_nan(fmax_nan(zd[4], zd[5]), fmax_nan(zd[6], zd[7])));
+        badD |= md != md || md == INFINITY;
         if (md > RD) {
           SD = RD == -INFINITY ? 0.f : SD * ex2((RD - md) * cT);
           RD = md;
@@ -215,12 +208,16 @@ __device__ __noinline__ void verify_pass1(VSmem& sm, const TIn* rT, const TIn* r
     }
   }
   {
-    float st = ST, sd = SD;
+    // the warp's pair from the lanes' pairs (a lane's reference is finite or -inf)
+    float MT = RT, MD = RD;
+    warp_max2(MT, MD);
+    float st = RT == -INFINITY ? 0.f : ST * ex2((RT - MT) * cT);
+    float sd = RD == -INFINITY ? 0.f : SD * ex2((RD - MD) * cT);
     warp_sum2(st, sd);
     if (lane == 0) {
-      sm.rm[0][warp] = RT;
+      sm.rm[0][warp] = MT;
       sm.rs[0][warp] = st;
-      sm.rm[1][warp] = RD;
+      sm.rm[1][warp] = MD;
       sm.rs[1][warp] = sd;
     }
     if (__any_sync(0xffffffffu, badT) && lane == 0) atomicOr(&sm.flag, 1);

@@ -13,11 +13,11 @@
 // does it, at HBM speed.
 //
 // Kernel: persistent CTAs of 512 threads (two per SM) take rows in turn.  A
-// warp takes tiles of 512 entries (16 per lane, two 16-byte loads of bf16,
-// two tiles in flight); every exp is relative to the warp's running max R
-// (one redux per tile, so no exp can overflow), and each lane parks the sum of
-// its 16 exps in shared memory with the tile's R.  Every 8 tiles the warp
-// scores their 32 blocks one per lane: the block's sum from its 8 lanes' partials, then
+// warp takes tiles of 1024 entries (32 per lane, four 16-byte loads of bf16);
+// every exp is relative to the warp's running max R (one redux per tile, so no
+// exp can overflow), and each lane parks the sum of its 32 exps in shared
+// memory with the tile's R.  Every 4 tiles the warp scores their 32 blocks one
+// per lane: the block's sum from its 4 lanes' partials, then
 // ln(sum) + R/tau + G_j with fp32 error bounds, folded into the row's (max,
 // sum) partial for the log-sum-exp.  The CTA merges the block candidates; a
 // block decision the fp32 bounds do not settle is redone in fp64 over the
@@ -32,11 +32,11 @@ namespace smcsd {
 
 constexpr int kDThreads = 512;  // 16 warps
 constexpr int kDBlk = 128;      // entries per block of the draw
-constexpr int kDBuf = 8;        // tiles a warp buffers before scoring their blocks
-constexpr int kDTile = 512;     // entries per warp tile: 16 per lane, four blocks
+constexpr int kDBuf = 4;        // tiles a warp buffers before scoring their blocks
+constexpr int kDTile = 1024;    // entries per warp tile: 32 per lane, eight blocks
 
 struct DraftSmem {
-  float part[kDThreads / 32][kDBuf][32];  // per lane: sum of its 16 exps, relative to the tile's R
+  float part[kDThreads / 32][kDBuf][32];  // per lane: sum of its 32 exps, relative to the tile's R
   float ref[kDThreads / 32][kDBuf];       // the tile's reference R (the warp's running max)
   int tile[kDThreads / 32][kDBuf];
   Cand cand[kDThreads / 32];
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kDThreads, 2) draft_block_kernel(
     const TIn* __restrict__ z, int rows, int V, int64_t ld, float inv_tau, float cT, double tau64,
     uint64_t seed, uint64_t round, uint32_t row0, int vec, int32_t* __restrict__ tokens_out,
     float* __restrict__ logq_out, uint32_t* dev_err) {
-  constexpr int kDUnroll = sizeof(TIn) == 2 ? 2 : 1;  // tiles in flight: 64 bytes a lane
+  constexpr int kDUnroll = 1;  // tiles in flight: 64 bytes a lane (bf16)
   __shared__ DraftSmem sm;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = kDThreads / 32;
@@ -82,11 +82,11 @@ __global__ void __launch_bounds__(kDThreads, 2) draft_block_kernel(
     // the block noise can span (< 20).
     auto score_blocks = [&]() {
       __syncwarp();
-      const int q = lane >> 2, h = lane & 3;  // lane: block h of buffered tile q
+      const int q = lane >> 3, h = lane & 7;  // lane: block h of buffered tile q
       if (q < nbuf) {
         float sb = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) sb += sm.part[warp][q][8 * h + i];
+        for (int i = 0; i < 4; ++i) sb += sm.part[warp][q][4 * h + i];
         const float rb = sm.ref[warp][q];
         if (sb > 0.f && sb < INFINITY) {
           if (rb > M) {
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kDThreads, 2) draft_block_kernel(
             M = rb;
           }
           S += sb * ex2((rb - M) * cT);
-          const int j = 4 * sm.tile[warp][q] + h;
+          const int j = 8 * sm.tile[warp][q] + h;
           const U4 w = sblk.at((uint32_t)(j >> 2), rid);
           const float g32 = gumbel_f32(uniform_f32(word_of(w, j & 3)));
           const float lam = logf(sb) + rb * inv_tau;
@@ -115,27 +115,29 @@ __global__ void __launch_bounds__(kDThreads, 2) draft_block_kernel(
       nbuf = 0;
     };
     for (int t0 = warp; t0 < nt; t0 += kDUnroll * nw) {
-      Raw8<TIn> raw[kDUnroll][2];
+      Raw8<TIn> raw[kDUnroll][4];
 #pragma unroll
       for (int u = 0; u < kDUnroll; ++u) {
         const int t = t0 + u * nw;
         if (t < nt) {
-          raw[u][0] = load8_raw<TIn>(row, t * kDTile + 16 * lane, V, vecok, pol);
-          raw[u][1] = load8_raw<TIn>(row, t * kDTile + 16 * lane + 8, V, vecok, pol);
+#pragma unroll
+          for (int h = 0; h < 4; ++h)
+            raw[u][h] = load8_raw<TIn>(row, t * kDTile + 32 * lane + 8 * h, V, vecok, pol);
         }
       }
 #pragma unroll
       for (int u = 0; u < kDUnroll; ++u) {
         const int t = t0 + u * nw;
         if (t >= nt) break;  // warp-uniform
-        float zz[16];
-        unpack8<TIn>(raw[u][0], zz);
-        unpack8<TIn>(raw[u][1], zz + 8);
-        float ma = fmax_nan(fmax_nan(fmax_nan(zz[0], zz[1]), fmax_nan(zz[2], zz[3])),
-                            fmax_nan(fmax_nan(zz[4], zz[5]), fmax_nan(zz[6], zz[7])));
-        float mb = fmax_nan(fmax_nan(fmax_nan(zz[8], zz[9]), fmax_nan(zz[10], zz[11])),
-                            fmax_nan(fmax_nan(zz[12], zz[13]), fmax_nan(zz[14], zz[15])));
-        const float m8 = fmax_nan(ma, mb);
+        float mq[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          float zz[8];
+          unpack8<TIn>(raw[u][h], zz);
+          mq[h] = fmax_nan(fmax_nan(fmax_nan(zz[0], zz[1]), fmax_nan(zz[2], zz[3])),
+                           fmax_nan(fmax_nan(zz[4], zz[5]), fmax_nan(zz[6], zz[7])));
+        }
+        const float m8 = fmax_nan(fmax_nan(mq[0], mq[1]), fmax_nan(mq[2], mq[3]));
         bad |= m8 != m8;
         float mt = m8 != m8 ? -INFINITY : m8;
         asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mt));
@@ -146,11 +148,16 @@ __global__ void __launch_bounds__(kDThreads, 2) draft_block_kernel(
           const float2 c2 = f2(cT), n2 = f2(-R * cT);
           float2 acc = f2(0.f), acc2 = f2(0.f);
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float2 ta = __ffma2_rn(make_float2(zz[i], zz[i + 1]), c2, n2);
-            const float2 tb = __ffma2_rn(make_float2(zz[i + 2], zz[i + 3]), c2, n2);
-            acc = __fadd2_rn(acc, make_float2(ex2(ta.x), ex2(ta.y)));
-            acc2 = __fadd2_rn(acc2, make_float2(ex2(tb.x), ex2(tb.y)));
+          for (int h = 0; h < 4; ++h) {
+            float zz[8];
+            unpack8<TIn>(raw[u][h], zz);
+#pragma unroll
+            for (int i = 0; i < 8; i += 4) {
+              const float2 ta = __ffma2_rn(make_float2(zz[i], zz[i + 1]), c2, n2);
+              const float2 tb = __ffma2_rn(make_float2(zz[i + 2], zz[i + 3]), c2, n2);
+              acc = __fadd2_rn(acc, make_float2(ex2(ta.x), ex2(ta.y)));
+              acc2 = __fadd2_rn(acc2, make_float2(ex2(tb.x), ex2(tb.y)));
+            }
           }
           sl = (acc.x + acc.y) + (acc2.x + acc2.y);
         }

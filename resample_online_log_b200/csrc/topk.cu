@@ -16,10 +16,10 @@
 // per-entry Gumbels have exactly this law, so the order is Gumbel-top-k's.
 //
 // Dense kernel (persistent CTAs, two per SM, each taking rows in turn):
-//   pass (HBM, once): a warp takes tiles of 512 entries (16 per lane, two
-//     tiles in flight); exps relative to the warp's running max R (one redux
-//     per tile); each lane parks the sum of its 16 exps with the tile's R;
-//     every 8 tiles the warp scores their 32 blocks, one per lane: M_j with
+//   pass (HBM, once): a warp takes tiles of 1024 entries (32 per lane, four
+//     16-byte loads of bf16); exps relative to the warp's running max R (one
+//     redux per tile); each lane parks the sum of its 32 exps with the tile's
+//     R; every 4 tiles the warp scores their 32 blocks, one per lane: M_j with
 //     fp32 error bounds into a per-row table, and the row's log-sum-exp partial;
 //   blocks: the k-th largest of the threads' best lower bounds is a lower
 //     bound T on the k-th largest M, so the blocks whose upper bound reaches T
@@ -39,14 +39,14 @@ constexpr int kTopkMax = 16;      // k <= 16 (also the sparse row length limit)
 constexpr int kTThreads = 512;    // 16 warps
 constexpr int kTWarps = kTThreads / 32;
 constexpr int kTBlk = 128;        // entries per block
-constexpr int kTBuf = 8;          // tiles a warp buffers before scoring their blocks
-constexpr int kTTile = 512;       // entries per warp tile: 16 per lane, four blocks
+constexpr int kTBuf = 4;          // tiles a warp buffers before scoring their blocks
+constexpr int kTTile = 1024;      // entries per warp tile: 32 per lane, eight blocks
 constexpr int kTMaxBlocks = 2048; // V <= 262144
 constexpr int kTCand = 256;       // candidate blocks gathered per row
 constexpr int kTEnt = kTopkMax * kTBlk;  // entries of the kept blocks
 
 struct TopkSmem {
-  float part[kTWarps][kTBuf][32];  // per lane: sum of its 16 exps, relative to the tile's R
+  float part[kTWarps][kTBuf][32];  // per lane: sum of its 32 exps, relative to the tile's R
   float ref[kTWarps][kTBuf];
   int tile[kTWarps][kTBuf];
   float bs[kTMaxBlocks];           // block maxima M_j (fp32), -inf: empty block
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kTThreads, 2) topk_block_kernel(
     const TIn* __restrict__ z, int rows, int V, int64_t ld, int k, float inv_tau, float cT,
     double tau64, uint64_t seed, uint64_t round, int vec, int32_t* __restrict__ idx_out,
     float* __restrict__ score_out, float* __restrict__ logp_out, uint32_t* dev_err) {
-  constexpr int kUnroll = sizeof(TIn) == 2 ? 2 : 1;  // tiles in flight: 64 bytes a lane
+  constexpr int kUnroll = 1;  // tiles in flight: 64 bytes a lane (bf16)
   extern __shared__ __align__(16) unsigned char topk_smem[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -282,13 +282,13 @@ __global__ void __launch_bounds__(kTThreads, 2) topk_block_kernel(
     int nbuf = 0;
     auto score_blocks = [&]() {
       __syncwarp();
-      const int q = lane >> 2, h = lane & 3;  // lane: block h of buffered tile q
+      const int q = lane >> 3, h = lane & 7;  // lane: block h of buffered tile q
       if (q < nbuf) {
         float sb = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) sb += sm.part[warp][q][8 * h + i];
+        for (int i = 0; i < 4; ++i) sb += sm.part[warp][q][4 * h + i];
         const float rb = sm.ref[warp][q];
-        const int j = 4 * sm.tile[warp][q] + h;
+        const int j = 8 * sm.tile[warp][q] + h;
         float mj = -INFINITY, dj = 0.f;
         if (sb > 0.f && sb < INFINITY) {
           if (rb > M) {
@@ -315,27 +315,29 @@ __global__ void __launch_bounds__(kTThreads, 2) topk_block_kernel(
       nbuf = 0;
     };
     for (int t0 = warp; t0 < nt; t0 += kUnroll * kTWarps) {
-      Raw8<TIn> raw[kUnroll][2];
+      Raw8<TIn> raw[kUnroll][4];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int t = t0 + u * kTWarps;
         if (t < nt) {
-          raw[u][0] = load8_raw<TIn>(row, t * kTTile + 16 * lane, V, vecok, pol);
-          raw[u][1] = load8_raw<TIn>(row, t * kTTile + 16 * lane + 8, V, vecok, pol);
+#pragma unroll
+          for (int h = 0; h < 4; ++h)
+            raw[u][h] = load8_raw<TIn>(row, t * kTTile + 32 * lane + 8 * h, V, vecok, pol);
         }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int t = t0 + u * kTWarps;
         if (t >= nt) break;  // warp-uniform
-        float zz[16];
-        unpack8<TIn>(raw[u][0], zz);
-        unpack8<TIn>(raw[u][1], zz + 8);
-        const float ma = fmax_nan(fmax_nan(fmax_nan(zz[0], zz[1]), fmax_nan(zz[2], zz[3])),
-                                  fmax_nan(fmax_nan(zz[4], zz[5]), fmax_nan(zz[6], zz[7])));
-        const float mb = fmax_nan(fmax_nan(fmax_nan(zz[8], zz[9]), fmax_nan(zz[10], zz[11])),
-                                  fmax_nan(fmax_nan(zz[12], zz[13]), fmax_nan(zz[14], zz[15])));
-        const float m8 = fmax_nan(ma, mb);
+        float mq[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          float zz[8];
+          unpack8<TIn>(raw[u][h], zz);
+          mq[h] = fmax_nan(fmax_nan(fmax_nan(zz[0], zz[1]), fmax_nan(zz[2], zz[3])),
+                           fmax_nan(fmax_nan(zz[4], zz[5]), fmax_nan(zz[6], zz[7])));
+        }
+        const float m8 = fmax_nan(fmax_nan(mq[0], mq[1]), fmax_nan(mq[2], mq[3]));
         bad |= m8 != m8;
         float mt = m8 != m8 ? -INFINITY : m8;
         asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(mt));
@@ -346,11 +348,16 @@ __global__ void __launch_bounds__(kTThreads, 2) topk_block_kernel(
           const float2 c2 = f2(cT), n2 = f2(-R * cT);
           float2 acc = f2(0.f), acc2 = f2(0.f);
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float2 ta = __ffma2_rn(make_float2(zz[i], zz[i + 1]), c2, n2);
-            const float2 tb = __ffma2_rn(make_float2(zz[i + 2], zz[i + 3]), c2, n2);
-            acc = __fadd2_rn(acc, make_float2(ex2(ta.x), ex2(ta.y)));
-            acc2 = __fadd2_rn(acc2, make_float2(ex2(tb.x), ex2(tb.y)));
+          for (int h = 0; h < 4; ++h) {
+            float zz[8];
+            unpack8<TIn>(raw[u][h], zz);
+#pragma unroll
+            for (int i = 0; i < 8; i += 4) {
+              const float2 ta = __ffma2_rn(make_float2(zz[i], zz[i + 1]), c2, n2);
+              const float2 tb = __ffma2_rn(make_float2(zz[i + 2], zz[i + 3]), c2, n2);
+              acc = __fadd2_rn(acc, make_float2(ex2(ta.x), ex2(ta.y)));
+              acc2 = __fadd2_rn(acc2, make_float2(ex2(tb.x), ex2(tb.y)));
+            }
           }
           sl = (acc.x + acc.y) + (acc2.x + acc2.y);
         }

@@ -67,9 +67,10 @@ __global__ void wait_kernel(uint64_t limit_ns, int mode, uint64_t delay_ns, uint
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const uint64_t t0 = globaltimer_ns();
+    // measured from t_start, the arriving warp's reference too, so that a wait
+    // ended by an arrival after delay_ns lasts at least delay_ns
     bounded_wait(&bar, 0u, &abort_flag, err, 1u << 8, (mode & 2) != 0, limit_ns);
-    out[0] = globaltimer_ns() - t0;
+    out[0] = globaltimer_ns() - t_start;
     out[1] = (uint64_t)abort_flag;
   } else if (threadIdx.x == 32 && (mode & 4)) {
     while (globaltimer_ns() - t_start < delay_ns) {

@@ -13,19 +13,20 @@
 // Design (B200, sm_100a).  Every (sequence, position) row is independent until
 // the first rejection is known, so all rows are scored at once:
 //   verify_rows_kernel: persistent CTAs of 512 threads (two per SM) take rows
-//     in turn, streaming each row twice in tiles of 256 entries (8 per lane,
-//     16-byte loads, several tiles in flight):
-//     pass 1 (HBM; the row stays in L2): the log-sum-exp of the target and
+//     in turn, streaming each row twice with 16-byte loads, several in flight:
+//     pass 1 (HBM, tiles of 256 entries, 8 per lane; the row stays in L2):
+//       the log-sum-exp of the target and
 //       draft rows, exps relative to each lane's running max (the warp
 //       combines its lanes once, after the row); the accept test
 //       u q(x) < p(x) in fp64;
-//     pass 2 (L2): p and q per entry, TV = 1/2 sum |p - q|, and the block
-//       masses the row's draw needs -- residual sum max(p - q, 0) after a
-//       rejection (with the error bound 7.7e-6 (p + q) per entry), target
-//       mass on the last row -- parked per lane and scored per block one per
-//       lane every 16 tiles; the CTA merges the block candidates (a near-tie,
-//       or no residual mass in fp32, goes to fp64 over the row's blocks), and
-//       one warp draws the entry inside the chosen block in fp64.
+//     pass 2 (L2, tiles of 512 entries: 16 per lane): p and q per entry,
+//       TV = 1/2 sum |p - q|, and the block masses the row's draw needs --
+//       residual sum max(p - q, 0) after a rejection (with the error bound
+//       7.7e-6 (p + q) per entry), target mass on the last row -- parked per
+//       lane and scored per block one per lane every 8 tiles; the CTA merges
+//       the block candidates (a near-tie, or no residual mass in fp32, goes to
+//       fp64 over the row's blocks), and one warp draws the entry inside the
+//       chosen block in fp64.
 //     Each row's outcome is encoded in its own slot of out_tokens.
 //   verify_finalize_kernel: per sequence, the first rejection decides the
 //     accepted length and the emitted tokens; slots past it become -1.
@@ -42,7 +43,8 @@ constexpr int kVThreads = 512;
 constexpr int kVPerSM = 2;
 constexpr int kVWarps = kVThreads / 32;
 constexpr int kVBlk = 128;
-constexpr int kVBuf = 16;  // tiles a warp buffers before scoring their blocks
+constexpr int kVBuf = 8;   // pass-2 tiles a warp buffers before scoring their blocks
+constexpr int kVTile2 = 512;  // pass-2 warp tile: 16 entries a lane, four blocks
 
 struct VerifyArgs {
   const void* zT;
@@ -61,8 +63,8 @@ struct VerifyArgs {
 };
 
 struct VSmem {
-  float part[kVWarps][kVBuf][32];  // per lane: its 8 entries' block mass (residual or target)
-  float pq[kVWarps][kVBuf][32];    // per lane: its 8 entries' p + q (residual error bounds)
+  float part[kVWarps][kVBuf][32];  // per lane: its 16 entries' block mass (residual or target)
+  float pq[kVWarps][kVBuf][32];    // per lane: its 16 entries' p + q (residual error bounds)
   int tile[kVWarps][kVBuf];
   float rm[2][kVWarps], rs[2][kVWarps];  // lse partials (target, draft)
   float tv[kVWarps];
@@ -233,24 +235,23 @@ __device__ __noinline__ void verify_pass2(VSmem& sm, const TIn* rT, const TIn* r
                                           bool hasD, int mode, bool badTr, bool badDr, float cT,
                                           float LT, float LD, bool vec, uint64_t drop,
                                           const Stream& sblk, uint32_t rid) {
-  constexpr int kUnroll = sizeof(TIn) == 2 ? 2 : 1;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float tvp = 0.f;
   Cand best = cand_empty();
   int nbuf = 0;
   auto score_blocks = [&]() {
     __syncwarp();
-    const int q = lane >> 1, h = lane & 1;  // lane: block h of buffered tile q
+    const int q = lane >> 2, h = lane & 3;  // lane: block h of buffered tile q
     if (q < nbuf) {
       float m = 0.f, e = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) m += sm.part[warp][q][16 * h + i];
+      for (int i = 0; i < 8; ++i) m += sm.part[warp][q][8 * h + i];
       if (mode == 1) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) e += sm.pq[warp][q][16 * h + i];
+        for (int i = 0; i < 8; ++i) e += sm.pq[warp][q][8 * h + i];
         e = 7.7e-6f * e + 1e-35f;  // |fp32 r - r| <= 7.7e-6 (p + q) per entry
       }
-      const int jb = 2 * sm.tile[warp][q] + h;
+      const int jb = 4 * sm.tile[warp][q] + h;
       if (m + e > 0.f) {
         const U4 w = sblk.at((uint32_t)(jb >> 2), rid);
         const float g32 = gumbel_f32(uniform_f32(word_of(w, jb & 3)));
@@ -281,24 +282,20 @@ __device__ __noinline__ void verify_pass2(VSmem& sm, const TIn* rT, const TIn* r
     nbuf = 0;
   };
   if (hasD || mode == 2) {
-    for (int t0 = warp; t0 < nt; t0 += kUnroll * kVWarps) {
-      Raw8<TIn> xt[kUnroll], xd[kUnroll];
+    const int nt2 = (V + kVTile2 - 1) / kVTile2;
+    for (int t = warp; t < nt2; t += kVWarps) {
+      Raw8<TIn> xt[2], xd[2];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int t = t0 + u * kVWarps;
-        if (t < nt) {
-          xt[u] = load8_raw<TIn>(rT, t * 256 + 8 * lane, V, vec, drop);
-          if (hasD) xd[u] = load8_raw<TIn>(rD, t * 256 + 8 * lane, V, vec, drop);
-        }
+      for (int u = 0; u < 2; ++u) {
+        xt[u] = load8_raw<TIn>(rT, t * kVTile2 + 16 * lane + 8 * u, V, vec, drop);
+        if (hasD) xd[u] = load8_raw<TIn>(rD, t * kVTile2 + 16 * lane + 8 * u, V, vec, drop);
       }
+      float bm = 0.f, bpq = 0.f;
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int t = t0 + u * kVWarps;
-        if (t >= nt) break;  // warp-uniform
+      for (int u = 0; u < 2; ++u) {
         float zt[8], zd[8];
         unpack8<TIn>(xt[u], zt);
         if (hasD) unpack8<TIn>(xd[u], zd);
-        float bm = 0.f, bpq = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float p = badTr ? 0.f : ex2(fmaf(zt[i], cT, -LT));
@@ -311,12 +308,12 @@ __device__ __noinline__ void verify_pass2(VSmem& sm, const TIn* rT, const TIn* r
             bm += p;
           }
         }
-        if (mode != 0) {
-          sm.part[warp][nbuf][lane] = bm;
-          if (mode == 1) sm.pq[warp][nbuf][lane] = bpq;
-          if (lane == 0) sm.tile[warp][nbuf] = t;
-          if (++nbuf == kVBuf) score_blocks();
-        }
+      }
+      if (mode != 0) {
+        sm.part[warp][nbuf][lane] = bm;
+        if (mode == 1) sm.pq[warp][nbuf][lane] = bpq;
+        if (lane == 0) sm.tile[warp][nbuf] = t;
+        if (++nbuf == kVBuf) score_blocks();
       }
     }
     if (mode != 0) score_blocks();
